@@ -1,0 +1,37 @@
+"""fp64 CPU oracle for ring-ordered blockwise attention.
+
+This package is TEST INFRASTRUCTURE. Only the test suite, the smoke check in
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it.
+The product path (the CUDA library and its Python binding) never calls it and
+shares no code with it: the two meet only through the seeded inputs.
+
+Every function cites the passage of the source pages it restates; the pages
+are
+
+* "Ring Attention 环注意力" (slowleelab, ai-terms-fun) -- the primary page,
+  cited by its layer and section (L3 definition, L4 §4.2 algorithm, §4.3
+  fusion with FlashAttention, §4.5 limitations, L5 §5.2 pitfalls);
+* the FlashAttention / PagedAttention article (developer.aliyun), section 二
+  (FlashAttention core principle, FlashAttention-2, FlashAttention-3);
+* "大模型底层原理注意力机制优化与长上下文处理" (lnwmold), §2.1 (standard
+  self-attention) and §2.2 (MQA/GQA).
+
+Every function here has a pin in ``tests/test_oracle.py`` against something
+other than itself (a library routine, a closed form, an invariant, the pages'
+worked example, or brute force on tiny inputs); none is parity unpinned.
+"""
+
+from .attn_fp64 import (  # noqa: F401
+    NEG_INF,
+    attention,
+    attention_rows,
+    attention_probs,
+    brute_attention,
+    ring_order,
+    ring_visits,
+    ring_attention,
+    ring_attention_merged,
+    merge,
+    causal_pair_counts,
+    kv_bytes_per_ring_step,
+)
