@@ -1,0 +1,353 @@
+#!/usr/bin/env python
+"""Benchmark of the ring-ordered attention forward on B200.
+
+One step = one ``ring_attn_fwd`` over the headline workload (causal, B=1,
+Hq=Hkv=32, L=131072, d=128, eight ring blocks of 16384 tokens), inputs
+already resident in HBM.  The inputs (3 GiB of bf16 Q/K/V) exceed the 126 MB
+L2, so no flush is needed between steps.
+
+``python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]``
+prints ONE JSON line on rank 0.  Under torchrun every rank runs its own copy
+of the workload (independent problems, no collective on the data path:
+weak scaling); timing is the max over ranks of the CUDA-event time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+method has) on a bounded sample of query rows of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s & % of B200 BF16 tensor peak (1 GPU), causal L=128K"
+UNIT = "TFLOP/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk["bf16_tflops_sustained"]),
+                "hbm_gbs": float(pk["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while the
+    timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_oracle_sample(w, budget_s: float, seed: int = 12345):
+    """Time the fp64 oracle on uniformly sampled query rows of the workload,
+    batches of 64 rows until ``budget_s`` of CPU time is spent.  Returns
+    (flops, seconds, rows, threads)."""
+    import numpy as np
+    import oracle
+    from ring_attention_ordered_b200.inputs import sample_rows, workload_inputs
+
+    q, k, v = workload_inputs(w)
+    rows = sample_rows(w, 1 << 16, seed=seed)
+    done, flops, t_used = 0, 0.0, 0.0
+    while t_used < budget_s and done < len(rows):
+        batch = rows[done:done + 64]
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.causal, w.scale, batch)
+        t_used += time.perf_counter() - t0
+        keys = (batch[:, 2] + 1) if w.causal else np.full(len(batch), w.L)
+        flops += float(4.0 * w.d * keys.sum())
+        done += len(batch)
+    return flops, t_used, done, os.cpu_count()
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return 0
+    os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count()))
+    per_step = []
+    total_flops = total_t = 0.0
+    rows = 0
+    threads = os.cpu_count()
+    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        fl, t, n, threads = cpu_oracle_sample(w, budget, seed=1000 + i)
+        if i >= args.warmup:
+            per_step.append(t)
+            total_flops += fl
+            total_t += t
+            rows += n
+    value = total_flops / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.describe(), "name": w.name},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} uniformly sampled query rows over {args.steps} steps"
+                                   f" (all their allowed keys), fp64 numpy"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    from ring_attention_ordered_b200 import _lib, api
+    from ring_attention_ordered_b200.inputs import workload_inputs
+
+    _lib.load()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+
+    peaks = load_peaks()
+    q_h, k_h, v_h = workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        api.fwd(q, k, v, w.n_ring, w.causal, w.scale, out=out, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    api.check_status(stream)
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    api.check_status(stream)
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    elapsed = ev[0].elapsed_time(ev[-1])
+    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_max = float(t.item())
+
+    flops = w.flops()
+    value = world * args.steps * flops / (elapsed_max / 1e3) / 1e12
+
+    # end to end: pinned host inputs -> device, forward, outputs -> pinned host
+    q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        q.copy_(q_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        step()
+        out_p.copy_(out, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    api.check_status(stream)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * e2e_steps * flops / (float(te.item()) / 1e3) / 1e12
+    h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+
+    # the merge kernel (the standalone fold of two partials), HBM-bound:
+    # 3 * (4d + 4) bytes per row over all rows of the workload
+    rows = w.B * w.Hq * w.L
+    o_a = torch.randn(rows, w.d, device=dev)
+    o_b = torch.randn(rows, w.d, device=dev)
+    l_a = torch.randn(rows, device=dev)
+    l_b = torch.randn(rows, device=dev)
+    o_o, l_o = torch.empty_like(o_a), torch.empty_like(l_a)
+    for _ in range(3):
+        api.merge(o_a, l_a, o_b, l_b, out=o_o, lse_out=l_o, stream=stream)
+    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    m0.record(stream)
+    for _ in range(reps):
+        api.merge(o_a, l_a, o_b, l_b, out=o_o, lse_out=l_o, stream=stream)
+    m1.record(stream)
+    torch.cuda.synchronize(dev)
+    merge_ms = m0.elapsed_time(m1) / reps
+    merge_bytes = 3 * (4 * w.d + 4) * rows
+    del o_a, o_b, l_a, l_b, o_o, l_o
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    avg_launch_ms = sum(per_launch) / len(per_launch)
+    achieved = flops / (avg_launch_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        fl, tcpu, nrows, threads = cpu_oracle_sample(w, args.cpu_budget)
+        cpu = {"value": fl / tcpu / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{nrows} uniformly sampled query rows of the workload with all their "
+                         f"allowed keys, fp64 numpy, {tcpu:.1f} s"}
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.describe(), "name": w.name, "global_batch": w.B * world,
+                   "seq_len": w.L, "parallelism": f"replicas{world}",
+                   "l2": "inputs (3 GiB) exceed L2; no flush",
+                   "flop_convention": "4*B*Hq*L^2*d / 2 (causal)"},
+        "frac_of_peak": {"of_burst": value / world / peaks["bf16_tflops"],
+                         "of_sustained": value / world / peaks["bf16_tflops_sustained"],
+                         "peaks": peaks["source"]},
+        "tokens_per_s": world * args.steps * w.B * w.L / (elapsed_max / 1e3),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "ra_fwd_kernel<128>",
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "merge": {"ms": merge_ms, "GB/s": merge_bytes / (merge_ms / 1e3) / 1e9,
+                  "frac_hbm": merge_bytes / (merge_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                  "rows": rows, "d": w.d},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    from ring_attention_ordered_b200.inputs import HEADLINE, WORKLOADS
+    w = WORKLOADS[args.workload or HEADLINE]
+    world, rank, local = dist_setup()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+    return run_ours(args, w, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,142 @@
+/*
+ * ring_attn.h -- C ABI of the B200 (sm_100a) ring-ordered blockwise attention
+ * library (libring_attn.so).
+ *
+ * The operation follows "Ring Attention 环注意力" (slowleelab, ai-terms-fun):
+ * the sequence of length L is cut into n_ring equal blocks (L4 §4.2 setup);
+ * the query block of host i visits the K/V blocks in ring order
+ * (i - t) mod n_ring for t = 0..n_ring-1 (L3 definition, L4 §4.2); every
+ * visit is exact blockwise attention whose partial result is folded into a
+ * running online-softmax accumulator (L4 §4.3), and under causal masking the
+ * later blocks are skipped (L4 §4.5, limitation 2).  The n_ring hosts are
+ * emulated as n_ring sequence blocks on one GPU; no data leaves the device.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never frees or retains them after the call returns.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream).  Argument errors are reported synchronously, before anything is
+ *     launched; device-side failures are reported by ring_attn_check_status.
+ *   - No C++ exception crosses the ABI.  A non-OK status leaves a one-line
+ *     explanation that ring_attn_last_error() returns (per host thread).
+ *   - The library holds no device allocation of its own except one status
+ *     word per device (a static device variable of the module).
+ */
+#ifndef RING_ATTN_H_
+#define RING_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* ra_stream_t;
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID_ARG = 1,  /* a shape, pointer, alignment or value is invalid   */
+  RA_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements  */
+  RA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                 */
+  RA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (see below)    */
+} ra_status;
+
+/*
+ * ring_attn_fwd -- forward ring-ordered blockwise attention.
+ *
+ * Computes, for every batch b, query head h and row r,
+ *     out[b, r, h, :] = sum_c softmax_c(scale * q[b,r,h,:] . k[b,c,h/g,:]) v[b,c,h/g,:]
+ *     lse[b, h, r]    = ln sum_c exp(scale * q[b,r,h,:] . k[b,c,h/g,:])
+ * over the keys c allowed by the mask (all c, or c <= r when causal), with
+ * g = Hq / Hkv query heads sharing one K/V head (grouped-query attention,
+ * lnwmold page §2.2; contiguous groups: head h reads K/V head h / g).  The
+ * work is organised as the ring of the pages: query block i visits K/V blocks
+ * (i - t) mod n_ring, t = 0..n_ring-1; causal visits with j > i are skipped,
+ * the j == i visit is masked on its diagonal, j < i visits run unmasked.
+ *
+ *   q      bf16 [B, L, Hq,  d], contiguous (d fastest)              (in)
+ *   k, v   bf16 [B, L, Hkv, d], contiguous                          (in)
+ *   out    bf16 [B, L, Hq,  d], contiguous, fp32-accumulated and
+ *          rounded to nearest even                                  (out)
+ *   lse    fp32 [B, Hq, L], contiguous, natural-log log-sum-exp     (out)
+ *   B, Hq, Hkv, L, d, n_ring   sizes; L % n_ring == 0 (equal blocks),
+ *          Hq % Hkv == 0, d in {64, 128}; any block length L/n_ring >= 1
+ *          (blocks that are not a multiple of 128 rows end in a partial
+ *          tile); B*L < 2^31.
+ *   causal 0 or 1
+ *   scale  finite and >= 0 (the pages use 1/sqrt(d); 0 gives uniform weights)
+ *
+ * Pointers must be 16-byte aligned and out/lse must not overlap the inputs.
+ * B*Hq*L == 0 is a valid empty problem: nothing is launched and the pointers
+ * may be NULL.
+ * Errors: RA_ERR_INVALID_ARG for the conditions above, RA_ERR_UNSUPPORTED for
+ * d outside {64, 128} or a device that is not compute capability 10.0,
+ * RA_ERR_CUDA if the launch fails.  Nothing is written on error.
+ */
+ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int Hq, int Hkv, int64_t L, int d, int n_ring, int causal,
+                        float scale, ra_stream_t stream);
+
+/*
+ * ring_attn_merge -- fold two partial attention results over disjoint key
+ * sets into one (the accumulation of each ring step's blockwise result into
+ * O_i, "Ring Attention 环注意力" L4 §4.2 step 2, kept as output plus
+ * logsumexp as in FlashAttention-2):
+ *     M = max(lse_a, lse_b), w = exp(lse - M)
+ *     lse_out = M + ln(w_a + w_b)
+ *     o_out   = (w_a o_a + w_b o_b) / (w_a + w_b)
+ * A partial with lse = -inf is empty: the other one is returned exactly (its
+ * o may hold anything, NaN included); two empty partials give o = 0 and
+ * lse = -inf.  NaN in an lse propagates to that row.  The result is bitwise
+ * identical when a and b are swapped.
+ *
+ *   o_a, o_b, o_out   fp32 [rows, d], contiguous
+ *   lse_a, lse_b, lse_out fp32 [rows]
+ *   rows >= 0, d >= 1 with d % 4 == 0; 16-byte aligned pointers.
+ * o_out/lse_out may be exactly o_a/lse_a or o_b/lse_b (in place); any other
+ * overlap is invalid.  rows == 0 launches nothing.
+ */
+ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b,
+                          const float* lse_b, float* o_out, float* lse_out, int64_t rows, int d,
+                          ra_stream_t stream);
+
+/*
+ * ring_attn_check_status -- synchronise `stream`, then read and clear the
+ * device status word of the current device.  Every device-side wait of the
+ * forward kernel is bounded (see ring_attn_set_wait_limit_ns); a wait that
+ * runs out makes the kernel record RA_ERR_TIMEOUT, release its tensor memory
+ * and return, leaving the CUDA context usable.  Returns RA_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+ra_status ring_attn_check_status(ra_stream_t stream);
+
+/* Longest any single device-side wait may take before the kernel gives up
+ * (nanoseconds; default 5e9).  0 restores the default.  Process-wide. */
+ra_status ring_attn_set_wait_limit_ns(uint64_t ns);
+
+/* Cap on the number of persistent CTAs of the forward kernel (0 = one per
+ * SM, the default).  Process-wide; used to exercise the scheduler. */
+ra_status ring_attn_set_max_ctas(int n);
+
+/* Host-side fault injection for tests.  Bit 0: the forward kernel's loader
+ * skips the first query-tile load, so the first bounded wait on it runs out
+ * and the call reports RA_ERR_TIMEOUT through ring_attn_check_status.
+ * 0 clears.  Process-wide. */
+ra_status ring_attn_debug_inject(unsigned flags);
+
+/* Human-readable name of a status code (static storage). */
+const char* ring_attn_status_string(ra_status s);
+
+/* Explanation of the last non-OK status returned on this host thread
+ * ("" if none).  Valid until the next call on the same thread. */
+const char* ring_attn_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int ring_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RING_ATTN_H_ */

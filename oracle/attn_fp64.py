@@ -35,6 +35,10 @@ NEG_INF = float("-inf")
 
 
 def _f64(x) -> np.ndarray:
+    # torch tensors (bf16 included) are widened through float32, which holds
+    # every bf16 value exactly
+    if hasattr(x, "detach") and hasattr(x, "float"):
+        x = x.detach().cpu().float().numpy()
     return np.asarray(x, dtype=np.float64)
 
 
@@ -122,7 +126,7 @@ def attention_rows(q, k, v, causal: bool, scale: float, bhr, row_block: int = 12
             sel = idx[s0:s0 + row_block]
             rs = bhr[sel, 2]
             nk = int(rs.max()) + 1 if causal else L
-            qq = _f64(q[b, rs, h, :])
+            qq = _f64(q[b, rs.tolist() if hasattr(q, "detach") else rs, h, :])
             s = scale * (qq @ kk_all[:nk].T)
             if causal:
                 s[np.arange(nk)[None, :] > rs[:, None]] = NEG_INF

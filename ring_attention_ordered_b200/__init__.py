@@ -1,0 +1,19 @@
+"""B200-native ring-ordered blockwise attention.
+
+The product is the C-ABI library ``libring_attn.so`` (kernels for sm_100a,
+declared in ``include/ring_attn.h``).  This package holds its sources
+(``csrc/``), the in-tree build (``build``), the ctypes binding (``_lib``), a
+torch-facing wrapper (``api``) that only marshals tensors into the C calls,
+and the seeded synthetic inputs (``inputs``).
+"""
+
+from ._lib import (  # noqa: F401
+    RingAttnError,
+    ring_attn_check_status,
+    ring_attn_debug_inject,
+    ring_attn_fwd,
+    ring_attn_merge,
+    ring_attn_set_max_ctas,
+    ring_attn_set_wait_limit_ns,
+    ring_attn_version,
+)

@@ -1,0 +1,75 @@
+"""Torch-facing wrapper: checks tensors, allocates outputs with torch and
+passes raw pointers plus the current CUDA stream to the C ABI.  All
+arithmetic happens in the library's kernels."""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _check_cuda(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: bool,
+        scale: float | None = None, out: torch.Tensor | None = None,
+        lse: torch.Tensor | None = None, stream=None):
+    """Ring-ordered attention forward.  q [B, L, Hq, d], k/v [B, L, Hkv, d]
+    (bf16, contiguous, on the GPU).  Returns (out bf16 [B, L, Hq, d],
+    lse fp32 [B, Hq, L]).  ``scale`` defaults to 1/sqrt(d)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_cuda(t, n, torch.bfloat16, 4)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, L, Hkv, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    _check_cuda(out, "out", torch.bfloat16, 4)
+    _check_cuda(lse, "lse", torch.float32, 3)
+    with torch.cuda.device(q.device):
+        _lib.ring_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           lse.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale,
+                           _stream_handle(stream))
+    return out, lse
+
+
+def merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,
+          out: torch.Tensor | None = None, lse_out: torch.Tensor | None = None, stream=None):
+    """Log-sum-exp merge of two partials: o [rows, d] fp32, lse [rows] fp32."""
+    _check_cuda(o_a, "o_a", torch.float32, 2)
+    _check_cuda(o_b, "o_b", torch.float32, 2)
+    _check_cuda(lse_a, "lse_a", torch.float32, 1)
+    _check_cuda(lse_b, "lse_b", torch.float32, 1)
+    rows, d = o_a.shape
+    if out is None:
+        out = torch.empty_like(o_a)
+    if lse_out is None:
+        lse_out = torch.empty_like(lse_a)
+    with torch.cuda.device(o_a.device):
+        _lib.ring_attn_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
+                             out.data_ptr(), lse_out.data_ptr(), rows, d, _stream_handle(stream))
+    return out, lse_out
+
+
+def check_status(stream=None):
+    with torch.cuda.device(torch.cuda.current_device()):
+        _lib.ring_attn_check_status(_stream_handle(stream))

@@ -1,0 +1,257 @@
+// C ABI of libring_attn: argument validation, TMA tensor-map construction,
+// work-unit planning and launches.  Declared in include/ring_attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "ra_internal.h"
+#include "ring_attn.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_wait_limit_ns{5000000000ull};
+std::atomic<int> g_max_ctas{0};
+std::atomic<unsigned> g_debug_flags{0u};
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+int g_cc_ok[kMaxDevices] = {0};  // 0 unknown, 1 yes, -1 no
+std::mutex g_mu;
+
+ra_status fail(ra_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+ra_status ok() {
+  g_last_error.clear();
+  return RA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Query SM count and compute capability of the current device once.
+ra_status device_info(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(RA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_cc_ok[dev] == 0) {
+    int major = 0, minor = 0, n = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return fail(RA_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    g_cc_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    g_sm_count[dev] = n;
+  }
+  if (g_cc_ok[dev] != 1)
+    return fail(RA_ERR_UNSUPPORTED, "this library is built for sm_100a (compute capability 10.0)");
+  *sms = g_sm_count[dev];
+  return RA_OK;
+}
+
+// Tensor map over a bf16 [B*L, H, d] array (d fastest): box {64, 1, 128},
+// 128-byte swizzle, out-of-range rows read as zero.
+ra_status make_map(CUtensorMap* map, const void* base, int H, long long rows, int d) {
+  auto enc = get_encode_fn();
+  if (!enc) return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return RA_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                        int Hq, int Hkv, int64_t L, int d, int n_ring, int causal, float scale,
+                        ra_stream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || L < 0)
+    return fail(RA_ERR_INVALID_ARG, "negative size (B=%d Hq=%d Hkv=%d L=%lld)", B, Hq, Hkv,
+                static_cast<long long>(L));
+  if (n_ring < 1) return fail(RA_ERR_INVALID_ARG, "n_ring must be >= 1 (got %d)", n_ring);
+  if (causal != 0 && causal != 1) return fail(RA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (!std::isfinite(scale) || scale < 0.f)
+    return fail(RA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (L % n_ring != 0)
+    return fail(RA_ERR_INVALID_ARG, "L=%lld does not split into %d equal blocks",
+                static_cast<long long>(L), n_ring);
+  if (Hkv == 0 && Hq != 0) return fail(RA_ERR_INVALID_ARG, "Hkv must be >= 1");
+  if (Hkv > 0 && Hq % Hkv != 0)
+    return fail(RA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(RA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (static_cast<long long>(B) * Hq * L == 0) return ok();
+  if (static_cast<long long>(B) * L >= (1ll << 31))
+    return fail(RA_ERR_INVALID_ARG, "B*L must be < 2^31");
+  if (!q || !k || !v || !out || !lse) return fail(RA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(RA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t nq = static_cast<size_t>(B) * L * Hq * d * 2;
+  const size_t nkv = static_cast<size_t>(B) * L * Hkv * d * 2;
+  const size_t nl = static_cast<size_t>(B) * Hq * L * 4;
+  if (overlaps(out, nq, q, nq) || overlaps(out, nq, k, nkv) || overlaps(out, nq, v, nkv) ||
+      overlaps(lse, nl, q, nq) || overlaps(lse, nl, k, nkv) || overlaps(lse, nl, v, nkv) ||
+      overlaps(out, nq, lse, nl))
+    return fail(RA_ERR_INVALID_ARG, "outputs overlap the inputs or each other");
+
+  int sms = 0;
+  ra_status st = device_info(&sms);
+  if (st != RA_OK) return st;
+
+  ra::FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const long long rows = static_cast<long long>(B) * L;
+  if ((st = make_map(&prm.tm_q, q, Hq, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_k, k, Hkv, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_v, v, Hkv, rows, d)) != RA_OK) return st;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.L = static_cast<int>(L);
+  prm.n_ring = n_ring;
+  prm.blk_len = static_cast<int>(L / n_ring);
+  prm.causal = causal;
+  prm.tiles_per_blk = (prm.blk_len + 127) / 128;
+  prm.pair_heads = prm.group >= 2 ? 1 : 0;
+  prm.head_slots = (prm.group + 1) / 2;
+  prm.pairs_per_blk = (prm.tiles_per_blk + 1) / 2;
+  if (prm.pair_heads)
+    prm.total_units = static_cast<long long>(B) * Hkv * prm.head_slots * n_ring * prm.tiles_per_blk;
+  else
+    prm.total_units = static_cast<long long>(B) * Hq * n_ring * prm.pairs_per_blk;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.wait_limit_ns = g_wait_limit_ns.load();
+  prm.debug_flags = g_debug_flags.load();
+
+  long long grid = sms;
+  const int cap = g_max_ctas.load();
+  if (cap > 0 && cap < grid) grid = cap;
+  if (grid > prm.total_units) grid = prm.total_units;
+  cudaError_t e = ra::launch_fwd(prm, d, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "forward launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b,
+                          const float* lse_b, float* o_out, float* lse_out, int64_t rows, int d,
+                          ra_stream_t stream) {
+  if (rows < 0) return fail(RA_ERR_INVALID_ARG, "rows must be >= 0");
+  if (d < 1 || d % 4 != 0) return fail(RA_ERR_INVALID_ARG, "d must be a positive multiple of 4");
+  if (rows == 0) return ok();
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out)
+    return fail(RA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o_out) || !aligned16(lse_a) ||
+      !aligned16(lse_b) || !aligned16(lse_out))
+    return fail(RA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t no = static_cast<size_t>(rows) * d * 4, nl = static_cast<size_t>(rows) * 4;
+  auto bad_alias = [&](const void* out, size_t n, const void* in) {
+    return out != in && overlaps(out, n, in, n);
+  };
+  if (bad_alias(o_out, no, o_a) || bad_alias(o_out, no, o_b) || bad_alias(lse_out, nl, lse_a) ||
+      bad_alias(lse_out, nl, lse_b) || overlaps(o_out, no, lse_out, nl) ||
+      overlaps(o_out, no, lse_a, nl) || overlaps(o_out, no, lse_b, nl) ||
+      overlaps(lse_out, nl, o_a, no) || overlaps(lse_out, nl, o_b, no))
+    return fail(RA_ERR_INVALID_ARG, "outputs may alias an input exactly but not overlap otherwise");
+  int sms = 0;
+  ra_status st = device_info(&sms);
+  if (st != RA_OK) return st;
+  cudaError_t e = ra::launch_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d, sms,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+ra_status ring_attn_check_status(ra_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  unsigned long long v = 0;
+  e = ra::read_and_clear_status(&v);
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (v == 0) return ok();
+  const unsigned code = static_cast<unsigned>(v >> 32);
+  const unsigned site = static_cast<unsigned>((v >> 16) & 0xFFFF);
+  const unsigned cta = static_cast<unsigned>(v & 0xFFFF);
+  return fail(static_cast<ra_status>(code), "device wait ran out (site %u, CTA %u)", site, cta);
+}
+
+ra_status ring_attn_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? 5000000000ull : ns);
+  return ok();
+}
+
+ra_status ring_attn_set_max_ctas(int n) {
+  if (n < 0) return fail(RA_ERR_INVALID_ARG, "max CTAs must be >= 0");
+  g_max_ctas.store(n);
+  return ok();
+}
+
+ra_status ring_attn_debug_inject(unsigned flags) {
+  if (flags & ~1u) return fail(RA_ERR_INVALID_ARG, "unknown debug flag bits 0x%x", flags & ~1u);
+  g_debug_flags.store(flags);
+  return ok();
+}
+
+const char* ring_attn_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_INVALID_ARG: return "RA_ERR_INVALID_ARG";
+    case RA_ERR_UNSUPPORTED: return "RA_ERR_UNSUPPORTED";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA";
+    case RA_ERR_TIMEOUT: return "RA_ERR_TIMEOUT";
+  }
+  return "RA_ERR_UNKNOWN";
+}
+
+const char* ring_attn_last_error(void) { return g_last_error.c_str(); }
+
+int ring_attn_version(void) { return 100; }
+
+}  // extern "C"

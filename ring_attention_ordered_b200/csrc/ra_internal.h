@@ -1,0 +1,41 @@
+// Internal declarations shared by the kernels and the C ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace ra {
+
+// Parameters of one forward launch.  The tensor maps describe q, k and v as
+// 3-D arrays {d, H, B*L} of bf16 (d fastest) with a box of {64, 1, 128}:
+// 64 head-dim columns (one 128-byte swizzle row) of 128 consecutive rows of
+// one head.
+struct FwdParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  __nv_bfloat16* out;
+  float* lse;
+  int B, Hq, Hkv, group;
+  int L, blk_len, n_ring, causal;
+  int tiles_per_blk;   // ceil(blk_len / 128)
+  int pair_heads;      // 1: a unit is two heads of one GQA group on the same rows
+  int head_slots;      // ceil(group / 2), when pair_heads
+  int pairs_per_blk;   // ceil(tiles_per_blk / 2), when !pair_heads
+  long long total_units;
+  float scale_log2;    // scale * log2(e)
+  unsigned long long wait_limit_ns;
+  unsigned debug_flags;
+};
+
+cudaError_t launch_fwd(const FwdParams& prm, int d, int grid, cudaStream_t stream);
+cudaError_t read_and_clear_status(unsigned long long* out);
+
+cudaError_t launch_merge(const float* o_a, const float* lse_a, const float* o_b,
+                         const float* lse_b, float* o_out, float* lse_out, long long rows, int d,
+                         int num_sms, cudaStream_t stream);
+
+}  // namespace ra

@@ -1,0 +1,132 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects invalid arguments before touching the device."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from ring_attention_ordered_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ring_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from ring_attention_ordered_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ring_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert "ring_attn_fwd" in names and "ring_attn_merge" in names
+    assert set(names) == set(_lib.SIGNATURES), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version(lib):
+    for code, name in enumerate(["RA_OK", "RA_ERR_INVALID_ARG", "RA_ERR_UNSUPPORTED",
+                                 "RA_ERR_CUDA", "RA_ERR_TIMEOUT"]):
+        assert _lib.status_string(code) == name
+    assert _lib.status_string(99) == "RA_ERR_UNKNOWN"
+    assert _lib.ring_attn_version() == 100
+
+
+# Fake, never-dereferenced device addresses: validation rejects these calls
+# before any CUDA call is made.
+A = 1 << 20
+Q, K, V, O, LSE = A, 2 * A * 64, 3 * A * 64, 4 * A * 64, 5 * A * 64
+
+
+def fwd_status(lib, **kw):
+    args = dict(q=Q, k=K, v=V, out=O, lse=LSE, B=1, Hq=2, Hkv=2, L=512, d=128, n_ring=4,
+                causal=1, scale=0.088)
+    args.update(kw)
+    return lib.ring_attn_fwd(args["q"], args["k"], args["v"], args["out"], args["lse"],
+                             args["B"], args["Hq"], args["Hkv"], args["L"], args["d"],
+                             args["n_ring"], args["causal"], args["scale"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(L=510), _lib.RA_ERR_INVALID_ARG),            # blocks would be unequal
+    (dict(n_ring=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(Hkv=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(B=-1), _lib.RA_ERR_INVALID_ARG),
+    (dict(causal=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.RA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), _lib.RA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), _lib.RA_ERR_INVALID_ARG),
+    (dict(d=96), _lib.RA_ERR_UNSUPPORTED),
+    (dict(d=256), _lib.RA_ERR_UNSUPPORTED),
+    (dict(q=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(lse=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(k=K + 8), _lib.RA_ERR_INVALID_ARG),           # not 16-byte aligned
+    (dict(out=Q + 64), _lib.RA_ERR_INVALID_ARG),        # output overlaps q
+    (dict(lse=O + 16), _lib.RA_ERR_INVALID_ARG),        # lse overlaps out
+    (dict(B=1, L=1 << 31, n_ring=1), _lib.RA_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_invalid_arguments(lib, kw, status):
+    assert fwd_status(lib, **kw) == status
+    assert _lib.last_error()
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(L=0), dict(Hq=0, Hkv=0)])
+def test_fwd_empty_problem_launches_nothing(lib, kw):
+    assert fwd_status(lib, q=0, k=0, v=0, out=0, lse=0, **kw) == _lib.RA_OK
+
+
+def merge_status(lib, rows=64, d=128, **kw):
+    p = dict(o_a=A, lse_a=2 * A, o_b=3 * A, lse_b=4 * A, o_out=5 * A, lse_out=6 * A)
+    p.update(kw)
+    return lib.ring_attn_merge(p["o_a"], p["lse_a"], p["o_b"], p["lse_b"], p["o_out"],
+                               p["lse_out"], rows, d, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(rows=-1), _lib.RA_ERR_INVALID_ARG),
+    (dict(d=6), _lib.RA_ERR_INVALID_ARG),
+    (dict(d=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(o_a=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(lse_b=4 * A + 4), _lib.RA_ERR_INVALID_ARG),
+    (dict(o_out=A + 16), _lib.RA_ERR_INVALID_ARG),     # partial overlap with o_a
+    (dict(lse_out=5 * A), _lib.RA_ERR_INVALID_ARG),    # lse_out inside o_out
+])
+def test_merge_rejects_invalid_arguments(lib, kw, status):
+    assert merge_status(lib, **kw) == status
+
+
+def test_merge_zero_rows_is_ok(lib):
+    assert merge_status(lib, rows=0, o_a=0, lse_a=0, o_b=0, lse_b=0, o_out=0, lse_out=0) == _lib.RA_OK
+
+
+def test_options_validate(lib):
+    assert lib.ring_attn_set_max_ctas(-1) == _lib.RA_ERR_INVALID_ARG
+    assert lib.ring_attn_set_max_ctas(0) == _lib.RA_OK
+    assert lib.ring_attn_debug_inject(2) == _lib.RA_ERR_INVALID_ARG
+    assert lib.ring_attn_debug_inject(0) == _lib.RA_OK
+    assert lib.ring_attn_set_wait_limit_ns(0) == _lib.RA_OK
+
+
+def test_python_binding_raises_on_error(lib):
+    with pytest.raises(_lib.RingAttnError) as ei:
+        _lib.ring_attn_fwd(Q, K, V, O, LSE, 1, 2, 2, 510, 128, 4, 1, 0.1, 0)
+    assert ei.value.status == _lib.RA_ERR_INVALID_ARG
+    assert "equal blocks" in str(ei.value)

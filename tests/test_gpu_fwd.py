@@ -1,0 +1,196 @@
+"""GPU parity of ring_attn_fwd (through the C ABI) against the fp64 oracle."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import compare, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ra():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from ring_attention_ordered_b200 import _lib, api
+    _lib.load()
+    return api
+
+
+def run(api, q, k, v, n_ring, causal, scale=None):
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out, lse = api.fwd(qd, kd, vd, n_ring, causal, scale)
+    api.check_status()
+    return out.cpu(), lse.cpu()
+
+
+def full_compare(api, q, k, v, n_ring, causal, scale=None, what=""):
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out, lse = run(api, q, k, v, n_ring, causal, scale)
+    o_ref, l_ref = oracle.attention(q, k, v, causal, scale)
+    return compare(out, lse, o_ref, l_ref, what)
+
+
+# (B, Hq, Hkv, L, d, n_ring, causal): several tiles, ring sizes 1..16, GQA
+# groups 1..4 (odd group included), ragged blocks (not a multiple of 128
+# rows, shorter than one tile), tiny and single-row sequences
+SMALL = [
+    (1, 1, 1, 128, 64, 1, False),
+    (1, 1, 1, 128, 128, 1, True),
+    (1, 2, 2, 512, 128, 4, True),
+    (1, 2, 2, 512, 128, 4, False),
+    (2, 4, 1, 768, 128, 3, True),
+    (1, 4, 2, 1024, 64, 2, True),
+    (1, 3, 1, 512, 128, 2, True),
+    (1, 6, 2, 256, 128, 1, False),
+    (1, 2, 2, 1536, 128, 6, True),
+    (1, 1, 1, 2048, 128, 16, True),
+    (1, 1, 1, 2048, 64, 16, False),
+    (1, 2, 1, 600, 128, 3, True),      # blocks of 200 rows: a full tile + 72
+    (2, 4, 2, 200, 64, 5, False),      # blocks of 40 rows
+    (1, 2, 2, 200, 128, 5, True),
+    (1, 1, 1, 1, 64, 1, False),        # one row
+    (1, 1, 1, 3, 128, 3, True),        # one row per block
+    (3, 2, 2, 384, 128, 2, True),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d,n_ring,causal", SMALL)
+def test_small_shapes(ra, B, Hq, Hkv, L, d, n_ring, causal):
+    from ring_attention_ordered_b200.inputs import make_inputs
+    q, k, v = make_inputs(B, Hq, Hkv, L, d, seed=B * 1000 + L + d + n_ring)
+    full_compare(ra, q, k, v, n_ring, causal, what=f"{(B, Hq, Hkv, L, d, n_ring, causal)}")
+
+
+def test_workload_l512_d64_noncausal(ra):
+    from ring_attention_ordered_b200.inputs import WORKLOADS, workload_inputs
+    w = WORKLOADS["l512_d64_noncausal"]
+    q, k, v = workload_inputs(w)
+    full_compare(ra, q, k, v, w.n_ring, w.causal, w.scale, w.name)
+
+
+def test_workload_l8k_h8_causal_all_rows(ra):
+    from ring_attention_ordered_b200.inputs import WORKLOADS, workload_inputs
+    w = WORKLOADS["l8k_h8_causal"]
+    q, k, v = workload_inputs(w)
+    full_compare(ra, q, k, v, w.n_ring, w.causal, w.scale, w.name)
+
+
+def boundary_rows(w, heads):
+    """Rows around every ring-block boundary and the sequence ends."""
+    rows = set()
+    lb = w.block_len
+    for i in range(w.n_ring + 1):
+        for r in (i * lb - 2, i * lb - 1, i * lb, i * lb + 1, i * lb + 127, i * lb + 128):
+            if 0 <= r < w.L:
+                rows.add(r)
+    return np.array([[b, h, r] for b in range(w.B) for h in heads for r in sorted(rows)],
+                    dtype=np.int64)
+
+
+@pytest.mark.parametrize("name,n_sample", [
+    ("l32k_gqa4_causal", 2048),
+    ("l128k_h32_causal", 1024),
+    ("l1m_gqa4_sink_causal", 512),
+])
+def test_workload_sampled_rows(ra, name, n_sample):
+    from ring_attention_ordered_b200.inputs import WORKLOADS, sample_rows, workload_inputs
+    w = WORKLOADS[name]
+    q, k, v = workload_inputs(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    out, lse = ra.fwd(qd, kd, vd, w.n_ring, w.causal, w.scale)
+    ra.check_status()
+    del qd, kd, vd
+    bhr = np.concatenate([sample_rows(w, n_sample),
+                          boundary_rows(w, [0, w.Hq - 1])])
+    o_ref, l_ref = oracle.attention_rows(q, k, v, w.causal, w.scale, bhr)
+    b, h, r = (torch.from_numpy(bhr[:, i]).cuda() for i in range(3))
+    o_g = out[b, r, h, :]
+    l_g = lse[b, h, r]
+    compare(o_g, l_g, o_ref, l_ref, name)
+
+
+def test_special_zero_query_and_zero_scale(ra):
+    from ring_attention_ordered_b200.inputs import make_inputs
+    q, k, v = make_inputs(1, 2, 1, 640, 128, seed=11)
+    zq = torch.zeros_like(q)
+    # Q = 0: every allowed key equally likely -> prefix means, lse = ln(r + 1)
+    out, lse = run(ra, zq, k, v, 5, True, 1.0 / math.sqrt(128))
+    vv = to_np(v)[0, :, 0, :]
+    pref = np.cumsum(vv, axis=0) / np.arange(1, 641)[:, None]
+    compare(out[0, :, 0, :], lse[0, 0], pref, np.log(np.arange(1, 641)), "q=0")
+    # scale = 0 gives the same uniform weights for any q
+    out2, lse2 = run(ra, q, k, v, 5, True, 0.0)
+    compare(out2[0, :, 1, :], lse2[0, 1], pref, np.log(np.arange(1, 641)), "scale=0")
+
+
+def test_special_causal_row0_and_constant_values(ra):
+    from ring_attention_ordered_b200.inputs import make_inputs
+    q, k, v = make_inputs(1, 2, 2, 512, 64, seed=12)
+    out, lse = run(ra, q, k, v, 4, True)
+    # causal row 0 of every ring block's first host sees key 0 only
+    np.testing.assert_array_equal(to_np(out[0, 0]), to_np(v[0, 0]))
+    # constant V reproduces V
+    cv = v[:, :1].expand_as(v).contiguous()
+    out2, _ = run(ra, q, k, cv, 4, False)
+    err = np.abs(to_np(out2) - to_np(cv)).max()
+    assert err <= 1e-2, err
+
+
+def test_deterministic_and_schedule_invariant(ra):
+    """The result does not depend on how many persistent CTAs share the work
+    (each unit is computed the same way whichever CTA takes it)."""
+    from ring_attention_ordered_b200 import _lib
+    from ring_attention_ordered_b200.inputs import make_inputs
+    q, k, v = make_inputs(2, 4, 2, 1024, 128, seed=13)
+    ref = run(ra, q, k, v, 4, True)
+    try:
+        for cap in (1, 3, 7, 0):
+            _lib.ring_attn_set_max_ctas(cap)
+            got = run(ra, q, k, v, 4, True)
+            assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1]), cap
+    finally:
+        _lib.ring_attn_set_max_ctas(0)
+
+
+def test_bounded_wait_reports_timeout_and_recovers(ra):
+    """A load that never comes makes the first bounded wait run out: the call
+    reports RA_ERR_TIMEOUT, the context stays usable and the next call is
+    correct (the aborted CTAs released their tensor memory)."""
+    from ring_attention_ordered_b200 import _lib
+    from ring_attention_ordered_b200.inputs import make_inputs
+    q, k, v = make_inputs(1, 2, 2, 512, 128, seed=14)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    try:
+        _lib.ring_attn_set_wait_limit_ns(200_000_000)
+        _lib.ring_attn_debug_inject(1)
+        ra.fwd(qd, kd, vd, 4, True)
+        with pytest.raises(_lib.RingAttnError) as ei:
+            ra.check_status()
+        assert ei.value.status == _lib.RA_ERR_TIMEOUT
+    finally:
+        _lib.ring_attn_debug_inject(0)
+        _lib.ring_attn_set_wait_limit_ns(0)
+    full_compare(ra, q, k, v, 4, True, what="after timeout")
+
+
+def test_invalid_arguments_on_device(ra):
+    from ring_attention_ordered_b200 import _lib
+    q = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty((1, 2, 256), dtype=torch.float32, device="cuda")
+    p = q.data_ptr()
+    with pytest.raises(_lib.RingAttnError) as ei:   # misaligned q
+        _lib.ring_attn_fwd(p + 2, p, p, out.data_ptr(), lse.data_ptr(), 1, 2, 2, 256, 128, 2, 1,
+                           0.1, 0)
+    assert ei.value.status == _lib.RA_ERR_INVALID_ARG
+    with pytest.raises(_lib.RingAttnError) as ei:   # output overlaps an input
+        _lib.ring_attn_fwd(p, p, p, p, lse.data_ptr(), 1, 2, 2, 256, 128, 2, 1, 0.1, 0)
+    assert ei.value.status == _lib.RA_ERR_INVALID_ARG
