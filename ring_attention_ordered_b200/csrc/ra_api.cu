@@ -163,10 +163,12 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   prm.pair_heads = prm.group >= 2 ? 1 : 0;
   prm.head_slots = (prm.group + 1) / 2;
   prm.pairs_per_blk = (prm.tiles_per_blk + 1) / 2;
-  if (prm.pair_heads)
-    prm.total_units = static_cast<long long>(B) * Hkv * prm.head_slots * n_ring * prm.tiles_per_blk;
-  else
-    prm.total_units = static_cast<long long>(B) * Hq * n_ring * prm.pairs_per_blk;
+  const long long units =
+      prm.pair_heads
+          ? static_cast<long long>(B) * Hkv * prm.head_slots * n_ring * prm.tiles_per_blk
+          : static_cast<long long>(B) * Hq * n_ring * prm.pairs_per_blk;
+  if (units >= (1ll << 31)) return fail(RA_ERR_INVALID_ARG, "problem too large (%lld work units)", units);
+  prm.total_units = static_cast<int>(units);
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.wait_limit_ns = g_wait_limit_ns.load();
   prm.debug_flags = g_debug_flags.load();

@@ -57,11 +57,32 @@ constexpr int WARP_MMA = 9;
 // softmax warpgroups take them.  The shares must add up to at most the launch
 // total, which the host checks before the first launch.
 constexpr int LAUNCH_REGS = 168;
-constexpr int SOFTMAX_REGS = 216;
-constexpr int CONTROL_REGS = 72;
+constexpr int SOFTMAX_REGS = 224;
+constexpr int CONTROL_REGS = 56;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
 constexpr float RESCALE_LOG2 = 8.0f;
+// Columns (out of 128) of each score row whose 2^x is evaluated with a
+// polynomial on the FMA pipe instead of the MUFU ex2 unit: at full tensor rate
+// one MUFU ex2 per score element would keep MUFU exactly as busy as the
+// tensor core, so part of the exponentials move to the otherwise idle FMA
+// pipe.
+#ifndef RA_EMU_COLS
+#define RA_EMU_COLS 0
+#endif
+constexpr int EMU_COLS = RA_EMU_COLS;
+static_assert(EMU_COLS % 2 == 0 && EMU_COLS >= 0 && EMU_COLS <= 128, "emulated columns");
+// Longest single hardware suspension inside one mbarrier try_wait (ns).
+#ifndef RA_WAIT_HINT_NS
+#define RA_WAIT_HINT_NS 1000000u
+#endif
+// Minimax (relative error) cubic for 2^f on [-1/2, 1/2], fitted by
+// csrc/fit_exp2_poly.py (Remez exchange); max relative error 7.5e-5 with
+// float32 Horner evaluation.
+constexpr float EXP2_C0 = 9.999280572e-01f;
+constexpr float EXP2_C1 = 6.932609677e-01f;
+constexpr float EXP2_C2 = 2.426111251e-01f;
+constexpr float EXP2_C3 = 5.517166853e-02f;
 constexpr float LN2 = 0.69314718055994530942f;
 
 // Device status word: 0 = ok, otherwise (code << 32) | where.
@@ -97,34 +118,34 @@ struct Unit {
   int n_kv;        // K/V tiles visited, in ring order
 };
 
-__device__ __forceinline__ Unit decode_unit(const FwdParams& p, long long u) {
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit x;
   const int tpb = p.tiles_per_blk;
   if (p.pair_heads) {
-    const long long per_tile = static_cast<long long>(p.B) * p.Hkv * p.head_slots;
-    const long long r = u / per_tile;
-    long long rem = u % per_tile;
-    const int gt = p.n_ring * tpb - 1 - static_cast<int>(r);   // longest first
+    const int per_tile = p.B * p.Hkv * p.head_slots;
+    const int r = u / per_tile;
+    int rem = u % per_tile;
+    const int gt = p.n_ring * tpb - 1 - r;   // longest first
     x.blk = gt / tpb;
     const int local = gt % tpb;
-    const int slot = static_cast<int>(rem % p.head_slots);
+    const int slot = rem % p.head_slots;
     rem /= p.head_slots;
-    x.kvh = static_cast<int>(rem % p.Hkv);
-    x.b = static_cast<int>(rem / p.Hkv);
+    x.kvh = rem % p.Hkv;
+    x.b = rem / p.Hkv;
     x.h[0] = x.kvh * p.group + 2 * slot;
     x.h[1] = x.h[0] + 1;
     x.valid1 = (2 * slot + 1) < p.group;
     x.qt[0] = x.qt[1] = local;
   } else {
-    const long long per_pair = static_cast<long long>(p.B) * p.Hq;
-    const long long r = u / per_pair;
-    const int bh = static_cast<int>(u % per_pair);
+    const int per_pair = p.B * p.Hq;
+    const int r = u / per_pair;
+    const int bh = u % per_pair;
     x.b = bh / p.Hq;
     x.h[0] = x.h[1] = bh % p.Hq;
     x.kvh = x.h[0] / p.group;
     const int ppb = p.pairs_per_blk;
-    x.blk = p.n_ring - 1 - static_cast<int>(r / ppb);
-    const int pr = ppb - 1 - static_cast<int>(r % ppb);
+    x.blk = p.n_ring - 1 - r / ppb;
+    const int pr = ppb - 1 - r % ppb;
     x.qt[0] = 2 * pr;
     x.qt[1] = 2 * pr + 1;
     x.valid1 = x.qt[1] < tpb;
@@ -134,28 +155,32 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, long long u) {
   return x;
 }
 
-// idx-th K/V tile of a unit: its ring block j (returned in jb) and its tile
-// index inside that block.  The unit's own block comes first (step t = 0),
-// then blocks (i - t) mod n_ring for t = 1, 2, ...; inside a block the tiles
-// run in ascending order, and under causal masking the own block stops at the
-// unit's last query tile.
-__device__ __forceinline__ int kv_tile_at(const FwdParams& p, const Unit& x, int idx, int& jb) {
-  const int tpb = p.tiles_per_blk;
-  const int ndiag = p.causal ? (x.qt_last + 1) : tpb;
-  if (idx < ndiag) {
+// K/V tiles of a unit in visit order.  The unit's own block comes first
+// (ring step t = 0), then blocks (i - t) mod n_ring for t = 1, 2, ...; inside
+// a block the tiles run in ascending order, and under causal masking the own
+// block stops at the unit's last query tile while later blocks are skipped.
+struct KvIter {
+  int jb;      // ring block of the current tile
+  int kl;      // tile index inside that block
+  int end;     // tiles of this block to visit
+  __device__ __forceinline__ void start(const FwdParams& p, const Unit& x) {
     jb = x.blk;
-    return idx;
+    kl = 0;
+    end = p.causal ? (x.qt_last + 1) : p.tiles_per_blk;
   }
-  const int r = idx - ndiag;
-  const int step = 1 + r / tpb;
-  jb = (x.blk - step + p.n_ring) % p.n_ring;
-  return r % tpb;
-}
+  __device__ __forceinline__ void next(const FwdParams& p) {
+    if (++kl == end) {
+      kl = 0;
+      jb = (jb == 0) ? p.n_ring - 1 : jb - 1;
+      end = p.tiles_per_blk;
+    }
+  }
+};
 
 // Static persistent schedule: in round k, CTA c takes unit k*G + c (k even)
 // or k*G + G-1-c (k odd).  Units are sorted longest first, so the snake keeps
 // the per-CTA totals within about one unit of each other.
-__device__ __forceinline__ long long unit_for_round(long long k, int G, int c) {
+__device__ __forceinline__ int unit_for_round(int k, int G, int c) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
@@ -177,11 +202,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ct
                                          uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, RA_WAIT_HINT_NS)) return true;
     if (*cx.abort) return false;
-    if ((++spins & 31u) == 0u && globaltimer_ns() - t0 > cx.limit_ns) {
+    if (globaltimer_ns() - t0 > cx.limit_ns) {
       record_timeout(cx, site);
       return false;
     }
@@ -206,46 +230,64 @@ struct Bars {
   __device__ __forceinline__ uint32_t o_free(int w) const { return o_free0 + 8u * w; }
 };
 
+// Bounded wait executed by a whole warp; the result is warp-uniform.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Ctl& cx,
+                                          uint32_t site) {
+  const bool ok = wait_bar(bar, parity, cx, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------ loader
+// The whole warp runs the control flow, so every address and coordinate is
+// warp-uniform (uniform registers); lane 0 alone issues the copies.
 template <int D>
 __device__ void loader_role(const FwdParams& p, const Bars& br, uint32_t smem_base, const Ctl& cx) {
   using C = Cfg<D>;
   constexpr int NBOX = D / BOX_COLS;
+  const bool leader = (threadIdx.x & 31) == 0;
+  const uint32_t lead = leader ? 1u : 0u;
   const int G = gridDim.x, c = blockIdx.x;
   uint32_t kv_it = 0, q_uses = 0;
   bool q_pending = false;
-  for (long long k = 0;; ++k) {
-    const long long u = unit_for_round(k, G, c);
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
     if (u >= p.total_units) break;
     const Unit x = decode_unit(p, u);
-    if (q_uses > 0 && !wait_bar(br.q_empty, (q_uses - 1) & 1u, cx, SITE_Q_EMPTY)) goto drain;
+    if (q_uses > 0 && !wait_warp(br.q_empty, (q_uses - 1) & 1u, cx, SITE_Q_EMPTY)) goto drain;
     if ((p.debug_flags & 1u) && q_uses == 0) {
       // fault injection: the first query tiles are never requested
     } else {
       const int nq = x.valid1 ? 2 : 1;
-      mbar_arrive_expect_tx(br.q_full, nq * C::Q_BYTES);
-      for (int w = 0; w < nq; ++w) {
-        const int row = x.b * p.L + x.blk * p.blk_len + x.qt[w] * BM;
+      mbar_arrive_expect_tx_if(br.q_full, nq * C::Q_BYTES, lead);
+      const int row0 = x.b * p.L + x.blk * p.blk_len;
+#pragma unroll
+      for (int bx = 0; bx < NBOX; ++bx)
+        tma_load_3d_if(smem_base + C::OFF_Q + bx * BOX_BYTES, &p.tm_q, br.q_full, bx * BOX_COLS,
+                       x.h[0], row0 + x.qt[0] * BM, lead);
+      if (x.valid1) {
+#pragma unroll
         for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d(smem_base + C::OFF_Q + w * C::Q_BYTES + bx * BOX_BYTES, &p.tm_q, br.q_full,
-                      bx * BOX_COLS, x.h[w], row);
+          tma_load_3d_if(smem_base + C::OFF_Q + C::Q_BYTES + bx * BOX_BYTES, &p.tm_q, br.q_full,
+                         bx * BOX_COLS, x.h[1], row0 + x.qt[1] * BM, lead);
       }
       q_pending = true;
     }
     ++q_uses;
-    for (int idx = 0; idx < x.n_kv; ++idx) {
-      int jb;
-      const int kl = kv_tile_at(p, x, idx, jb);
-      const int row = x.b * p.L + jb * p.blk_len + kl * BN;
+    KvIter it;
+    it.start(p, x);
+    for (int idx = 0; idx < x.n_kv; ++idx, it.next(p)) {
+      const int row = x.b * p.L + it.jb * p.blk_len + it.kl * BN;
+#pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int s = kv_it % C::NS;
         const uint32_t ph = (kv_it / C::NS) & 1u;
-        if (!wait_bar(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
-        mbar_arrive_expect_tx(br.kv_full(s), C::KV_BYTES);
+        if (!wait_warp(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
+        mbar_arrive_expect_tx_if(br.kv_full(s), C::KV_BYTES, lead);
         const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
+#pragma unroll
         for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d(smem_base + C::OFF_KV + s * C::KV_BYTES + bx * BOX_BYTES, map, br.kv_full(s),
-                      bx * BOX_COLS, x.kvh, row);
+          tma_load_3d_if(smem_base + C::OFF_KV + s * C::KV_BYTES + bx * BOX_BYTES, map,
+                         br.kv_full(s), bx * BOX_COLS, x.kvh, row, lead);
         ++kv_it;
       }
     }
@@ -253,7 +295,7 @@ __device__ void loader_role(const FwdParams& p, const Bars& br, uint32_t smem_ba
   return;
 drain:
   // Let the copies already issued land before the CTA's shared memory goes.
-  {
+  if (leader) {
     const uint32_t n = kv_it < static_cast<uint32_t>(C::NS) ? kv_it : C::NS;
     for (uint32_t i = 0; i < n; ++i) {
       const uint32_t it = kv_it - 1 - i;
@@ -261,109 +303,235 @@ drain:
     }
     if (q_pending) drain_wait(br.q_full, (q_uses - 1) & 1u, 200000000ull);
   }
+  __syncwarp();
 }
 
 // ------------------------------------------------------------------ MMA
+template <int KK>
+struct QkStep {
+  static constexpr uint32_t OFF = ((KK / 4) * BOX_BYTES + (KK % 4) * 32) >> 4;
+};
+
+// S = Q K^T over the head dimension: D/16 MMAs of K = 16.
+template <int D>
+__device__ __forceinline__ void mma_qk_steps(uint32_t d, uint32_t a, uint32_t b, uint32_t hi,
+                                             uint32_t idesc, uint32_t lead) {
+  mma_ss<QkStep<0>::OFF, QkStep<0>::OFF>(d, a, hi, b, hi, idesc, 0u, lead);
+  mma_ss<QkStep<1>::OFF, QkStep<1>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+  mma_ss<QkStep<2>::OFF, QkStep<2>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+  mma_ss<QkStep<3>::OFF, QkStep<3>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+  if constexpr (D == 128) {
+    mma_ss<QkStep<4>::OFF, QkStep<4>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+    mma_ss<QkStep<5>::OFF, QkStep<5>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+    mma_ss<QkStep<6>::OFF, QkStep<6>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+    mma_ss<QkStep<7>::OFF, QkStep<7>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+  }
+}
+
+// O (+)= P V over 128 keys: 8 MMAs of K = 16; P's 16 keys are 8 TMEM
+// columns of bf16 pairs, V's 16 keys are 16 rows of 128 bytes (2048 bytes).
+__device__ __forceinline__ void mma_pv_steps(uint32_t d, uint32_t p_tmem, uint32_t b, uint32_t hi,
+                                             uint32_t idesc, uint32_t acc, uint32_t lead) {
+  mma_ts<0, 0>(d, p_tmem, b, hi, idesc, acc, lead);
+  mma_ts<8, 128>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<16, 256>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<24, 384>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<32, 512>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<40, 640>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<48, 768>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<56, 896>(d, p_tmem, b, hi, idesc, 1u, lead);
+}
+
+// Warp-wide control flow as in the loader; lane 0 issues tcgen05.mma and
+// tcgen05.commit (a commit tracks the MMAs of the thread that issues it, so
+// both always come from lane 0).  Keeping descriptors warp-uniform lets
+// them live in uniform registers, which tcgen05.mma takes as operands.
 template <int D>
 __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base, uint32_t tmem,
                          const Ctl& cx) {
   using C = Cfg<D>;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
+  const bool leader = (threadIdx.x & 31) == 0;
   const int G = gridDim.x, c = blockIdx.x;
   uint32_t kv_it = 0, q_uses = 0;
-  uint32_t pf_phase[2] = {0u, 0u};
-  uint32_t units_w[2] = {0u, 0u};
+  uint32_t pf_phase0 = 0u, pf_phase1 = 0u;
+  uint32_t units0 = 0u, units1 = 0u;
 
-  // Descriptor start addresses are in 16-byte units in the low 14 bits; all
-  // shared-memory offsets here stay below 2^18 bytes, so adding (offset >> 4)
-  // to a base descriptor never carries out of that field.
+  // Shared-memory descriptors as (low, high) words.  The start address sits
+  // in the low 14 bits in 16-byte units; every offset used here keeps the
+  // address below 2^18 bytes, so adding (offset >> 4) to the low word never
+  // carries out of that field.  The high words are fixed by the layout.
   const uint64_t dq0 = smem_desc_sw128(smem_base + C::OFF_Q, 16, 1024);
   const uint64_t dkv0 = smem_desc_sw128(smem_base + C::OFF_KV, 16, 1024);
   const uint64_t dv0 = smem_desc_sw128(smem_base + C::OFF_KV, BOX_BYTES, 1024);
+  const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dkv0);
+  const uint32_t v_lo = static_cast<uint32_t>(dv0);
+  const uint32_t k_hi = static_cast<uint32_t>(dkv0 >> 32), v_hi = static_cast<uint32_t>(dv0 >> 32);
+  const uint32_t lead = leader ? 1u : 0u;
   auto issue_qk = [&](int w, int stage) {
-    const uint64_t dq = dq0 + static_cast<uint32_t>((w * C::Q_BYTES) >> 4);
-    const uint64_t dk = dkv0 + static_cast<uint32_t>((stage * C::KV_BYTES) >> 4);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = ((kk / 4) * BOX_BYTES + (kk % 4) * 32) >> 4;
-      mma_ss(tmem + w * 128, dq + off, dk + off, IDESC_QK, kk > 0 ? 1u : 0u);
-    }
+    const uint32_t a = q_lo + ((w * C::Q_BYTES) >> 4);
+    const uint32_t b = k_lo + ((stage * C::KV_BYTES) >> 4);
+    const uint32_t d = tmem + w * 128;
+    // k-steps of 16 elements: 32 bytes apart inside a 64-column swizzle
+    // box, the next box BOX_BYTES further on
+    mma_qk_steps<D>(d, a, b, k_hi, IDESC_QK, lead);
   };
   auto issue_pv = [&](int w, int stage, bool acc) {
-    const uint64_t dv = dv0 + static_cast<uint32_t>((stage * C::KV_BYTES) >> 4);
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-      mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + static_cast<uint32_t>(kk * 128),
-             IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-    }
+    const uint32_t b = v_lo + ((stage * C::KV_BYTES) >> 4);
+    mma_pv_steps(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u, lead);
   };
+  auto commit = [&](uint32_t bar) { tc_commit_if(bar, lead); };
 
-  for (long long k = 0;; ++k) {
-    const long long u = unit_for_round(k, G, c);
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
     if (u >= p.total_units) break;
     const Unit x = decode_unit(p, u);
     const int n = x.n_kv;
-    if (!wait_bar(br.q_full, q_uses & 1u, cx, SITE_Q_FULL)) goto drain;
+    if (!wait_warp(br.q_full, q_uses & 1u, cx, SITE_Q_FULL)) goto drain;
     tc_fence_after();
     ++q_uses;
     {
       const int ks = kv_it % C::NS;
-      if (!wait_bar(br.kv_full(ks), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+      if (!wait_warp(br.kv_full(ks), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
       tc_fence_after();
       issue_qk(0, ks);
-      tc_commit(br.s_full(0));
+      commit(br.s_full(0));
       if (x.valid1) {
         issue_qk(1, ks);
-        tc_commit(br.s_full(1));
+        commit(br.s_full(1));
       }
-      tc_commit(br.kv_empty(ks));
+      commit(br.kv_empty(ks));
       ++kv_it;
-      if (n == 1) tc_commit(br.q_empty);
+      if (n == 1) commit(br.q_empty);
     }
     for (int idx = 0; idx < n; ++idx) {
       const bool more = idx + 1 < n;
       const int vs = kv_it % C::NS;
       const int ks = (kv_it + 1) % C::NS;
-      if (!wait_bar(br.kv_full(vs), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+      if (!wait_warp(br.kv_full(vs), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
       tc_fence_after();
-      for (int w = 0; w < 2; ++w) {
-        if (w == 1 && !x.valid1) break;
-        if (!wait_bar(br.p_full(w), pf_phase[w], cx, SITE_P_FULL)) goto drain;
-        pf_phase[w] ^= 1u;
+      // query tile 0: P0 V, then S0 for the next K/V tile
+      if (!wait_warp(br.p_full(0), pf_phase0, cx, SITE_P_FULL)) goto drain;
+      pf_phase0 ^= 1u;
+      tc_fence_after();
+      if (idx == 0 && units0 > 0) {
+        if (!wait_warp(br.o_free(0), (units0 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
         tc_fence_after();
-        if (idx == 0 && units_w[w] > 0) {
-          if (!wait_bar(br.o_free(w), (units_w[w] - 1) & 1u, cx, SITE_O_FREE)) goto drain;
+      }
+      issue_pv(0, vs, idx > 0);
+      if (!more) commit(br.o_done(0));
+      if (more) {
+        if (!wait_warp(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+        tc_fence_after();
+        issue_qk(0, ks);
+        commit(br.s_full(0));
+      }
+      // query tile 1
+      if (x.valid1) {
+        if (!wait_warp(br.p_full(1), pf_phase1, cx, SITE_P_FULL)) goto drain;
+        pf_phase1 ^= 1u;
+        tc_fence_after();
+        if (idx == 0 && units1 > 0) {
+          if (!wait_warp(br.o_free(1), (units1 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
           tc_fence_after();
         }
-        issue_pv(w, vs, idx > 0);
-        if (!more) tc_commit(br.o_done(w));
+        issue_pv(1, vs, idx > 0);
+        if (!more) commit(br.o_done(1));
         if (more) {
-          if (w == 0) {
-            if (!wait_bar(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
-            tc_fence_after();
-          }
-          issue_qk(w, ks);
-          tc_commit(br.s_full(w));
+          issue_qk(1, ks);
+          commit(br.s_full(1));
         }
       }
-      tc_commit(br.kv_empty(vs));
+      commit(br.kv_empty(vs));
       if (more) {
-        tc_commit(br.kv_empty(ks));
-        if (idx + 1 == n - 1) tc_commit(br.q_empty);
+        commit(br.kv_empty(ks));
+        if (idx + 1 == n - 1) commit(br.q_empty);
       }
       kv_it += more ? 2u : 1u;
     }
-    ++units_w[0];
-    if (x.valid1) ++units_w[1];
+    ++units0;
+    if (x.valid1) ++units1;
   }
   return;
 drain:
-  tc_commit(br.drain);
-  drain_wait(br.drain, 0u, 200000000ull);
+  commit(br.drain);
+  if (leader) drain_wait(br.drain, 0u, 200000000ull);
+  __syncwarp();
 }
 
 // ------------------------------------------------------------------ softmax
+// 2^x for two values at once on the FMA pipe: x = j + f with j = round(x)
+// (adding and subtracting 1.5 * 2^23 rounds to the nearest integer), p(f) by
+// the cubic above, then 2^j applied by adding j << 23 to the bits of p(f)
+// (the low bits of x + 1.5 * 2^23 hold j in two's complement).  Inputs are
+// clamped to >= -125 so the scaled result stays a normal float; anything
+// below 2^-125 is negligible next to the row maximum's 2^0.
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  x2 = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t neg_magic = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t t = f2_add(x2, magic);
+  const uint64_t j = f2_add(t, neg_magic);
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x2);
+  uint64_t q = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
+  q = f2_fma(q, f, f2_pack(EXP2_C1, EXP2_C1));
+  q = f2_fma(q, f, f2_pack(EXP2_C0, EXP2_C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  r0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// One score row (128 columns held in sr): P = 2^(s * c2 - m) written as bf16
+// pairs to TMEM columns [0, 64) at tS, returns the row sum of the fp32 P.
+// MASKED: columns > lim are excluded (set to zero exactly).  Issues
+// warp-collective tcgen05.st: every lane of the warp must call the same
+// instantiation at the same time.
+template <bool MASKED>
+__device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, float m, int lim,
+                                               uint32_t tS) {
+  const uint64_t c2x2 = f2_pack(c2, c2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int col = 64 * half + 2 * j;
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])),
+                                 c2x2, nm2);
+      float p0, p1;
+      if (col < EMU_COLS) {
+        exp2_poly2(x2, p0, p1);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      if (MASKED) {
+        p0 = (col > lim) ? 0.f : p0;
+        p1 = (col + 1 > lim) ? 0.f : p1;
+      }
+      acc[j & 3] = f2_add(acc[j & 3], f2_pack(p0, p1));
+      pk[j] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32(tS + 32 * half, pk);
+  }
+  const uint64_t s01 = f2_add(acc[0], acc[1]);
+  const uint64_t s23 = f2_add(acc[2], acc[3]);
+  float a, b;
+  f2_unpack(f2_add(s01, s23), a, b);
+  return a + b;
+}
+
 template <int D>
 __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, int w,
                              const Ctl& cx) {
@@ -376,19 +544,19 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
   const int G = gridDim.x, cta = blockIdx.x;
   uint32_t s_phase = 0u, units_w = 0u;
 
-  for (long long k = 0;; ++k) {
-    const long long u = unit_for_round(k, G, cta);
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, cta);
     if (u >= p.total_units) break;
     const Unit x = decode_unit(p, u);
     if (w == 1 && !x.valid1) continue;
-    const int qt = x.qt[w];
-    const int h = x.h[w];
+    const int qt = w ? x.qt[1] : x.qt[0];
+    const int h = w ? x.h[1] : x.h[0];
     const int qrow = qt * BM + t;                  // row inside the ring block
     float m = -INFINITY, l = 0.f;
+    KvIter it;
+    it.start(p, x);
 
-    for (int idx = 0; idx < x.n_kv; ++idx) {
-      int jb;
-      const int kl = kv_tile_at(p, x, idx, jb);
+    for (int idx = 0; idx < x.n_kv; ++idx, it.next(p)) {
       bool ok = wait_bar(br.s_full(w), s_phase, cx, SITE_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) return;
       s_phase ^= 1u;
@@ -403,25 +571,24 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
       tmem_wait_ld();
 
       // keys allowed for this row: columns 0..lim of the tile
-      int lim = min(BN, p.blk_len - kl * BN) - 1;
-      if (p.causal && jb == x.blk) lim = min(lim, qrow - kl * BN);
-      const bool masked = lim < BN - 1;
-
-      float mx[8];
+      int lim = min(BN, p.blk_len - it.kl * BN) - 1;
+      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * BN);
+      // Warp-uniform: both branches below issue warp-collective tcgen05.st,
+      // which all 32 lanes must execute together.  Lanes whose own row needs
+      // no mask (lim = 127) run the masked code harmlessly.
+      const bool masked = __any_sync(0xffffffffu, lim < BN - 1);
+      if (masked) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-      if (!masked) {
-#pragma unroll
-        for (int j = 0; j < 128; ++j) mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sr[j]));
-      } else {
-#pragma unroll
-        for (int j = 0; j < 128; ++j) {
+        for (int j = 0; j < 128; ++j)
           if (j > lim) sr[j] = __float_as_uint(-INFINITY);
-          mx[j & 7] = fmaxf(mx[j & 7], __uint_as_float(sr[j]));
-        }
       }
-      float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      float mx[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 64; ++j)
+        mx[j & 3] = fmax3(mx[j & 3], __uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_tile = (rmax == -INFINITY) ? -INFINITY : rmax * c2;
       const bool need = m_tile > m + RESCALE_LOG2;
       const float m_new = need ? m_tile : m;
@@ -441,30 +608,9 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
         tmem_wait_st();
       }
       m = m_new;
-      l *= alpha;
-
-      const float neg_m = -m;
-      float rs[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) rs[i] = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int c0 = 64 * half + 2 * j;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sr[c0]), c2, neg_m));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sr[c0 + 1]), c2, neg_m));
-          if (masked) {
-            p0 = (c0 > lim) ? 0.f : p0;
-            p1 = (c0 + 1 > lim) ? 0.f : p1;
-          }
-          rs[j & 7] += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + 32 * half, pk);
-      }
-      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      const float rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS)
+                                : exp_row_store<false>(sr, c2, m, lim, tS);
+      l = l * alpha + rsum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(br.p_full(w));
@@ -566,9 +712,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_fwd_kernel(const __grid_con
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(CONTROL_REGS));
     if (warp == WARP_LOAD) {
-      if (lane == 0) loader_role<D>(p, br, base, cx);
+      loader_role<D>(p, br, base, cx);
     } else if (warp == WARP_MMA) {
-      if (lane == 0) mma_role<D>(p, br, base, tmem, cx);
+      mma_role<D>(p, br, base, tmem, cx);
     }
   }
 

@@ -25,7 +25,7 @@ struct FwdParams {
   int pair_heads;      // 1: a unit is two heads of one GQA group on the same rows
   int head_slots;      // ceil(group / 2), when pair_heads
   int pairs_per_blk;   // ceil(tiles_per_blk / 2), when !pair_heads
-  long long total_units;
+  int total_units;     // < 2^31, checked by the host
   float scale_log2;    // scale * log2(e)
   unsigned long long wait_limit_ns;
   unsigned debug_flags;
