@@ -90,7 +90,7 @@ __device__ unsigned long long g_ra_status = 0ull;
 
 enum WaitSite : uint32_t {
   SITE_Q_FULL = 1, SITE_Q_EMPTY, SITE_KV_FULL, SITE_KV_EMPTY, SITE_S_FULL,
-  SITE_P_FULL, SITE_O_DONE, SITE_O_FREE
+  SITE_P_FULL, SITE_O_DONE, SITE_O_FREE, SITE_P_HALF
 };
 
 template <int D>
@@ -102,8 +102,9 @@ struct Cfg {
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
   // barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2],
-  // p_full[2], o_done[2], o_free[2], drain; then tmem holder + abort flag
-  static constexpr int NUM_BARS = 2 + 2 * NS + 8 + 1;
+  // p_full[2], o_done[2], o_free[2], p_half[2], drain; then tmem holder +
+  // abort flag
+  static constexpr int NUM_BARS = 2 + 2 * NS + 10 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -221,13 +222,14 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 }
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, o_done0, o_free0, drain;
+  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, o_done0, o_free0, p_half0, drain;
   __device__ __forceinline__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
   __device__ __forceinline__ uint32_t kv_empty(int s) const { return kv_empty0 + 8u * s; }
   __device__ __forceinline__ uint32_t s_full(int w) const { return s_full0 + 8u * w; }
   __device__ __forceinline__ uint32_t p_full(int w) const { return p_full0 + 8u * w; }
   __device__ __forceinline__ uint32_t o_done(int w) const { return o_done0 + 8u * w; }
   __device__ __forceinline__ uint32_t o_free(int w) const { return o_free0 + 8u * w; }
+  __device__ __forceinline__ uint32_t p_half(int w) const { return p_half0 + 8u * w; }
 };
 
 // Bounded wait executed by a whole warp; the result is warp-uniform.
@@ -328,24 +330,20 @@ __device__ __forceinline__ void mma_qk_steps(uint32_t d, uint32_t a, uint32_t b,
   }
 }
 
-// O (+)= P V over 128 keys: 8 MMAs of K = 16; P's 16 keys are 8 TMEM
-// columns of bf16 pairs, V's 16 keys are 16 rows of 128 bytes (2048 bytes).
-__device__ __forceinline__ void mma_pv_steps(uint32_t d, uint32_t p_tmem, uint32_t b, uint32_t hi,
-                                             uint32_t idesc, uint32_t acc, uint32_t lead) {
-  mma_ts<0, 0>(d, p_tmem, b, hi, idesc, acc, lead);
-  mma_ts<8, 128>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<16, 256>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<24, 384>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<32, 512>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<40, 640>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<48, 768>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<56, 896>(d, p_tmem, b, hi, idesc, 1u, lead);
+// O (+)= P V over one half of the 128 keys (HALF 0: keys 0-63, 1: keys
+// 64-127): 4 MMAs of K = 16; P's 16 keys are 8 TMEM columns of bf16 pairs,
+// V's 16 keys are 16 rows of 128 bytes (2048 bytes).  `acc` applies to the
+// first MMA of the first half only.
+template <int HALF>
+__device__ __forceinline__ void mma_pv_half(uint32_t d, uint32_t p_tmem, uint32_t b, uint32_t hi,
+                                            uint32_t idesc, uint32_t acc, uint32_t lead) {
+  constexpr uint32_t C0 = 32 * HALF, B0 = 512 * HALF;
+  mma_ts<C0 + 0, B0 + 0>(d, p_tmem, b, hi, idesc, HALF ? 1u : acc, lead);
+  mma_ts<C0 + 8, B0 + 128>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<C0 + 16, B0 + 256>(d, p_tmem, b, hi, idesc, 1u, lead);
+  mma_ts<C0 + 24, B0 + 384>(d, p_tmem, b, hi, idesc, 1u, lead);
 }
 
-// Warp-wide control flow as in the loader; lane 0 issues tcgen05.mma and
-// tcgen05.commit (a commit tracks the MMAs of the thread that issues it, so
-// both always come from lane 0).  Keeping descriptors warp-uniform lets
-// them live in uniform registers, which tcgen05.mma takes as operands.
 template <int D>
 __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base, uint32_t tmem,
                          const Ctl& cx) {
@@ -377,9 +375,12 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
     // box, the next box BOX_BYTES further on
     mma_qk_steps<D>(d, a, b, k_hi, IDESC_QK, lead);
   };
-  auto issue_pv = [&](int w, int stage, bool acc) {
+  auto issue_pv_half = [&](int w, int stage, int half, bool acc) {
     const uint32_t b = v_lo + ((stage * C::KV_BYTES) >> 4);
-    mma_pv_steps(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u, lead);
+    if (half == 0)
+      mma_pv_half<0>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u, lead);
+    else
+      mma_pv_half<1>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, 1u, lead);
   };
   auto commit = [&](uint32_t bar) { tc_commit_if(bar, lead); };
 
@@ -410,33 +411,40 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
       const int vs = kv_it % C::NS;
       const int ks = (kv_it + 1) % C::NS;
       if (!wait_warp(br.kv_full(vs), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+      // the next K tile is needed right after P0 V: wait for it now, off the
+      // softmax -> MMA -> softmax chain
+      if (more && !wait_warp(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL))
+        goto drain;
       tc_fence_after();
-      // query tile 0: P0 V, then S0 for the next K/V tile
+      // query tile 0: P0 V in two halves as P0 arrives, then S0 for the next
+      // K/V tile
+      if (idx == 0 && units0 > 0) {
+        if (!wait_warp(br.o_free(0), (units0 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
+      }
+      if (!wait_warp(br.p_half(0), pf_phase0, cx, SITE_P_HALF)) goto drain;
+      tc_fence_after();
+      issue_pv_half(0, vs, 0, idx > 0);
       if (!wait_warp(br.p_full(0), pf_phase0, cx, SITE_P_FULL)) goto drain;
       pf_phase0 ^= 1u;
       tc_fence_after();
-      if (idx == 0 && units0 > 0) {
-        if (!wait_warp(br.o_free(0), (units0 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
-        tc_fence_after();
-      }
-      issue_pv(0, vs, idx > 0);
+      issue_pv_half(0, vs, 1, true);
       if (!more) commit(br.o_done(0));
       if (more) {
-        if (!wait_warp(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
-        tc_fence_after();
         issue_qk(0, ks);
         commit(br.s_full(0));
       }
       // query tile 1
       if (x.valid1) {
+        if (idx == 0 && units1 > 0) {
+          if (!wait_warp(br.o_free(1), (units1 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
+        }
+        if (!wait_warp(br.p_half(1), pf_phase1, cx, SITE_P_HALF)) goto drain;
+        tc_fence_after();
+        issue_pv_half(1, vs, 0, idx > 0);
         if (!wait_warp(br.p_full(1), pf_phase1, cx, SITE_P_FULL)) goto drain;
         pf_phase1 ^= 1u;
         tc_fence_after();
-        if (idx == 0 && units1 > 0) {
-          if (!wait_warp(br.o_free(1), (units1 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
-          tc_fence_after();
-        }
-        issue_pv(1, vs, idx > 0);
+        issue_pv_half(1, vs, 1, true);
         if (!more) commit(br.o_done(1));
         if (more) {
           issue_qk(1, ks);
@@ -488,12 +496,13 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1) {
 
 // One score row (128 columns held in sr): P = 2^(s * c2 - m) written as bf16
 // pairs to TMEM columns [0, 64) at tS, returns the row sum of the fp32 P.
+// Arrives on p_half_bar once the first 64 keys of P are stored.
 // MASKED: columns > lim are excluded (set to zero exactly).  Issues
 // warp-collective tcgen05.st: every lane of the warp must call the same
 // instantiation at the same time.
 template <bool MASKED>
 __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, float m, int lim,
-                                               uint32_t tS) {
+                                               uint32_t tS, uint32_t p_half_bar) {
   const uint64_t c2x2 = f2_pack(c2, c2);
   const uint64_t nm2 = f2_pack(-m, -m);
   uint64_t acc[4];
@@ -524,6 +533,12 @@ __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, fl
       pk[j] = pack_bf16x2(p0, p1);
     }
     tmem_st32(tS + 32 * half, pk);
+    if (half == 0) {
+      // the first 64 keys of P are in TMEM: let the MMA start on them
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_half_bar);
+    }
   }
   const uint64_t s01 = f2_add(acc[0], acc[1]);
   const uint64_t s23 = f2_add(acc[2], acc[3]);
@@ -557,59 +572,75 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
     it.start(p, x);
 
     for (int idx = 0; idx < x.n_kv; ++idx, it.next(p)) {
+      // keys allowed for this row: columns 0..lim of the tile.  Warp-uniform
+      // `masked`: both exp_row_store instantiations issue warp-collective
+      // tcgen05.st, which all 32 lanes must execute together; lanes whose own
+      // row needs no mask (lim = 127) run the masked code harmlessly.
+      int lim = min(BN, p.blk_len - it.kl * BN) - 1;
+      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * BN);
+      const bool masked = __any_sync(0xffffffffu, lim < BN - 1);
+
       bool ok = wait_bar(br.s_full(w), s_phase, cx, SITE_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) return;
       s_phase ^= 1u;
       tc_fence_after();
 
+      // S in two halves: the max over the first 64 columns runs while the
+      // second half is still being read from TMEM
       uint32_t sr[128];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[cc * 32]);
-        tmem_ld32(tS + cc * 32, chunk);
-      }
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
-
-      // keys allowed for this row: columns 0..lim of the tile
-      int lim = min(BN, p.blk_len - it.kl * BN) - 1;
-      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * BN);
-      // Warp-uniform: both branches below issue warp-collective tcgen05.st,
-      // which all 32 lanes must execute together.  Lanes whose own row needs
-      // no mask (lim = 127) run the masked code harmlessly.
-      const bool masked = __any_sync(0xffffffffu, lim < BN - 1);
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       if (masked) {
 #pragma unroll
-        for (int j = 0; j < 128; ++j)
+        for (int j = 0; j < 64; ++j)
           if (j > lim) sr[j] = __float_as_uint(-INFINITY);
       }
-      float mx[4];
+      float mx[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) mx[i] = -INFINITY;
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 64; ++j)
-        mx[j & 3] = fmax3(mx[j & 3], __uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
-      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      const float m_tile = (rmax == -INFINITY) ? -INFINITY : rmax * c2;
-      const bool need = m_tile > m + RESCALE_LOG2;
-      const float m_new = need ? m_tile : m;
-      const float alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
-      if (idx > 0 && __any_sync(0xffffffffu, need)) {
-        // O already holds every earlier P V of this tile: the commit that
-        // signalled S for this step fires only after them.
+      for (int j = 0; j < 32; ++j)
+        mx[j & 7] = fmax3(mx[j & 7], __uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+      tmem_wait_ld();
+      if (masked) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tO + cc * 32, o);
-        }
-        tmem_wait_st();
+        for (int j = 64; j < 128; ++j)
+          if (j > lim) sr[j] = __float_as_uint(-INFINITY);
       }
-      m = m_new;
-      const float rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS)
-                                : exp_row_store<false>(sr, c2, m, lim, tS);
+#pragma unroll
+      for (int j = 32; j < 64; ++j)
+        mx[j & 7] = fmax3(mx[j & 7], __uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float m_tile = (rmax == -INFINITY) ? -INFINITY : rmax * c2;
+      // Lazy rescale: move the reference max only when the tile max exceeds
+      // it by more than 2^8 (the final O / l cancels a stale max exactly).
+      const bool need = m_tile > m + RESCALE_LOG2;
+      float alpha = 1.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? m_tile : m;
+        alpha = (m_new == m) ? 1.f : ex2_approx(m - m_new);
+        if (idx > 0) {
+          // O already holds every earlier P V of this tile: the commit that
+          // signalled S for this step fires only after them.
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+          tmem_wait_st();
+        }
+        m = m_new;
+      }
+      const float rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS, br.p_half(w))
+                                : exp_row_store<false>(sr, c2, m, lim, tS, br.p_half(w));
       l = l * alpha + rsum;
       tmem_wait_st();
       tc_fence_before();
@@ -668,7 +699,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_fwd_kernel(const __grid_con
   br.p_full0 = br.s_full0 + 16;
   br.o_done0 = br.p_full0 + 16;
   br.o_free0 = br.o_done0 + 16;
-  br.drain = br.o_free0 + 16;
+  br.p_half0 = br.o_free0 + 16;
+  br.drain = br.p_half0 + 16;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::OFF_MISC + 4);
 
@@ -686,6 +718,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_fwd_kernel(const __grid_con
       mbar_init(br.p_full(w), 128);
       mbar_init(br.o_done(w), 1);
       mbar_init(br.o_free(w), 128);
+      mbar_init(br.p_half(w), 128);
     }
     mbar_init(br.drain, 1);
     *abort_flag = 0u;
