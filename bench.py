@@ -107,6 +107,35 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd.cu",
+                  "ring_attention_ordered_b200/csrc/ptx_sm100.cuh",
+                  "ring_attention_ordered_b200/csrc/ra_api.cu",
+                  "ring_attention_ordered_b200/csrc/ra_internal.h"]
+TRAFFIC_RECORD = "profiles/ra_fwd_l128k_h32_causal_dram.md"
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu record, or None when the
+    workload differs or the kernel sources changed since the capture."""
+    import hashlib
+    import re
+    if workload_name != "l128k_h32_causal":
+        return None
+    try:
+        text = open(os.path.join(ROOT, TRAFFIC_RECORD)).read()
+        h = hashlib.sha256()
+        for f in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    m_b = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    m_h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m_b or not m_h or m_h.group(1) != h.hexdigest():
+        return None
+    return int(m_b.group(1))
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -313,7 +342,7 @@ def run_ours(args, w, world, rank, local):
                          "peaks": peaks["source"]},
         "tokens_per_s": world * args.steps * w.B * w.L / (elapsed_max / 1e3),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name),
                      "kernel": "ra_fwd_kernel<128>",
                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})"},
         "cpu_baseline": cpu,

@@ -119,6 +119,18 @@ ra_status ring_attn_set_wait_limit_ns(uint64_t ns);
  * SM, the default).  Process-wide; used to exercise the scheduler. */
 ra_status ring_attn_set_max_ctas(int n);
 
+/* Order in which the forward kernel's persistent CTAs take work units (a unit
+ * = two 128-row query tiles sharing one K/V stream; causal units differ in
+ * length).  Results do not depend on it.  Process-wide.
+ *   RA_SCHEDULE_AUTO (default): HEAD_MAJOR when the K/V tensors exceed
+ *     256 MiB, else LONGEST_FIRST.
+ *   RA_SCHEDULE_LONGEST_FIRST: every unit sorted by length, longest first
+ *     (causal load balance, "Ring Attention 环注意力" L4 §4.5 limitation 3).
+ *   RA_SCHEDULE_HEAD_MAJOR: longest first within each (batch, K/V head), heads
+ *     one after another, so concurrently running CTAs share K/V tiles in L2. */
+enum { RA_SCHEDULE_AUTO = 0, RA_SCHEDULE_LONGEST_FIRST = 1, RA_SCHEDULE_HEAD_MAJOR = 2 };
+ra_status ring_attn_set_schedule(int schedule);
+
 /* Host-side fault injection for tests.  Bit 0: the forward kernel's loader
  * skips the first query-tile load, so the first bounded wait on it runs out
  * and the call reports RA_ERR_TIMEOUT through ring_attn_check_status.

@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     ring_attn_fwd,
     ring_attn_merge,
     ring_attn_set_max_ctas,
+    ring_attn_set_schedule,
     ring_attn_set_wait_limit_ns,
     ring_attn_version,
 )

@@ -27,6 +27,7 @@ SIGNATURES = {
     "ring_attn_check_status": (_I, [_P]),
     "ring_attn_set_wait_limit_ns": (_I, [ctypes.c_uint64]),
     "ring_attn_set_max_ctas": (_I, [_I]),
+    "ring_attn_set_schedule": (_I, [_I]),
     "ring_attn_debug_inject": (_I, [ctypes.c_uint]),
     "ring_attn_status_string": (ctypes.c_char_p, [_I]),
     "ring_attn_last_error": (ctypes.c_char_p, []),
@@ -92,6 +93,13 @@ def ring_attn_set_wait_limit_ns(ns: int):
 
 def ring_attn_set_max_ctas(n: int):
     return _check(load().ring_attn_set_max_ctas(n))
+
+
+RA_SCHEDULE_AUTO, RA_SCHEDULE_LONGEST_FIRST, RA_SCHEDULE_HEAD_MAJOR = 0, 1, 2
+
+
+def ring_attn_set_schedule(schedule: int):
+    return _check(load().ring_attn_set_schedule(schedule))
 
 
 def ring_attn_debug_inject(flags: int):

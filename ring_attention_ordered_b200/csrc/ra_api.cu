@@ -22,6 +22,12 @@ thread_local std::string g_last_error;
 std::atomic<unsigned long long> g_wait_limit_ns{5000000000ull};
 std::atomic<int> g_max_ctas{0};
 std::atomic<unsigned> g_debug_flags{0u};
+// Work-unit order: RA_SCHEDULE_AUTO picks K/V-head-major order when the K/V
+// tensors are much larger than L2 (CTAs then share one or two K/V heads at a
+// time, which stay L2-resident), else global longest-first order (best load
+// balance when K/V fits L2 anyway).
+std::atomic<int> g_schedule{RA_SCHEDULE_AUTO};
+constexpr double kHeadMajorKvBytes = 256.0 * 1024 * 1024;
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
@@ -169,6 +175,9 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
           : static_cast<long long>(B) * Hq * n_ring * prm.pairs_per_blk;
   if (units >= (1ll << 31)) return fail(RA_ERR_INVALID_ARG, "problem too large (%lld work units)", units);
   prm.total_units = static_cast<int>(units);
+  const int sched = g_schedule.load();
+  prm.head_major = sched == RA_SCHEDULE_HEAD_MAJOR ||
+                   (sched == RA_SCHEDULE_AUTO && 2.0 * static_cast<double>(nkv) > kHeadMajorKvBytes);
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.wait_limit_ns = g_wait_limit_ns.load();
   prm.debug_flags = g_debug_flags.load();
@@ -232,6 +241,14 @@ ra_status ring_attn_set_wait_limit_ns(uint64_t ns) {
 ra_status ring_attn_set_max_ctas(int n) {
   if (n < 0) return fail(RA_ERR_INVALID_ARG, "max CTAs must be >= 0");
   g_max_ctas.store(n);
+  return ok();
+}
+
+ra_status ring_attn_set_schedule(int schedule) {
+  if (schedule != RA_SCHEDULE_AUTO && schedule != RA_SCHEDULE_LONGEST_FIRST &&
+      schedule != RA_SCHEDULE_HEAD_MAJOR)
+    return fail(RA_ERR_INVALID_ARG, "unknown schedule %d", schedule);
+  g_schedule.store(schedule);
   return ok();
 }
 

@@ -119,14 +119,28 @@ struct Unit {
   int n_kv;        // K/V tiles visited, in ring order
 };
 
+// Unit order.  head_major = 0: all units sorted longest first across every
+// (batch, head).  head_major = 1: (batch, K/V head) major, longest first
+// inside each K/V head, so the CTAs running at any moment share one or two
+// K/V heads whose tiles stay in L2 instead of streaming from HBM.
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   Unit x;
   const int tpb = p.tiles_per_blk;
   if (p.pair_heads) {
-    const int per_tile = p.B * p.Hkv * p.head_slots;
-    const int r = u / per_tile;
-    int rem = u % per_tile;
-    const int gt = p.n_ring * tpb - 1 - r;   // longest first
+    const int n_tiles = p.n_ring * tpb;
+    int r, rem;
+    if (p.head_major) {
+      const int per_head = n_tiles * p.head_slots;
+      rem = u / per_head;                       // b * Hkv + kvh
+      const int v = u % per_head;
+      r = v / p.head_slots;
+      rem = rem * p.head_slots + v % p.head_slots;
+    } else {
+      const int per_tile = p.B * p.Hkv * p.head_slots;
+      r = u / per_tile;
+      rem = u % per_tile;
+    }
+    const int gt = n_tiles - 1 - r;   // longest first
     x.blk = gt / tpb;
     const int local = gt % tpb;
     const int slot = rem % p.head_slots;
@@ -138,9 +152,16 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     x.valid1 = (2 * slot + 1) < p.group;
     x.qt[0] = x.qt[1] = local;
   } else {
-    const int per_pair = p.B * p.Hq;
-    const int r = u / per_pair;
-    const int bh = u % per_pair;
+    int r, bh;
+    if (p.head_major) {
+      const int per_head = p.n_ring * p.pairs_per_blk;
+      bh = u / per_head;
+      r = u % per_head;
+    } else {
+      const int per_pair = p.B * p.Hq;
+      r = u / per_pair;
+      bh = u % per_pair;
+    }
     x.b = bh / p.Hq;
     x.h[0] = x.h[1] = bh % p.Hq;
     x.kvh = x.h[0] / p.group;

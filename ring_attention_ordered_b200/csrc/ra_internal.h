@@ -26,6 +26,7 @@ struct FwdParams {
   int head_slots;      // ceil(group / 2), when pair_heads
   int pairs_per_blk;   // ceil(tiles_per_blk / 2), when !pair_heads
   int total_units;     // < 2^31, checked by the host
+  int head_major;      // unit order: 1 = K/V-head major (L2 reuse), 0 = global longest first
   float scale_log2;    // scale * log2(e)
   unsigned long long wait_limit_ns;
   unsigned debug_flags;

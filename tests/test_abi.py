@@ -123,6 +123,9 @@ def test_options_validate(lib):
     assert lib.ring_attn_debug_inject(2) == _lib.RA_ERR_INVALID_ARG
     assert lib.ring_attn_debug_inject(0) == _lib.RA_OK
     assert lib.ring_attn_set_wait_limit_ns(0) == _lib.RA_OK
+    assert lib.ring_attn_set_schedule(3) == _lib.RA_ERR_INVALID_ARG
+    for sched in (_lib.RA_SCHEDULE_LONGEST_FIRST, _lib.RA_SCHEDULE_HEAD_MAJOR, _lib.RA_SCHEDULE_AUTO):
+        assert lib.ring_attn_set_schedule(sched) == _lib.RA_OK
 
 
 def test_python_binding_raises_on_error(lib):

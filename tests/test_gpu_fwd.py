@@ -146,18 +146,22 @@ def test_special_causal_row0_and_constant_values(ra):
 
 def test_deterministic_and_schedule_invariant(ra):
     """The result does not depend on how many persistent CTAs share the work
-    (each unit is computed the same way whichever CTA takes it)."""
+    or in which order they take the units (each unit is computed the same way
+    whichever CTA takes it, whenever)."""
     from ring_attention_ordered_b200 import _lib
     from ring_attention_ordered_b200.inputs import make_inputs
     q, k, v = make_inputs(2, 4, 2, 1024, 128, seed=13)
     ref = run(ra, q, k, v, 4, True)
     try:
-        for cap in (1, 3, 7, 0):
-            _lib.ring_attn_set_max_ctas(cap)
-            got = run(ra, q, k, v, 4, True)
-            assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1]), cap
+        for sched in (_lib.RA_SCHEDULE_LONGEST_FIRST, _lib.RA_SCHEDULE_HEAD_MAJOR):
+            _lib.ring_attn_set_schedule(sched)
+            for cap in (1, 3, 7, 0):
+                _lib.ring_attn_set_max_ctas(cap)
+                got = run(ra, q, k, v, 4, True)
+                assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1]), (sched, cap)
     finally:
         _lib.ring_attn_set_max_ctas(0)
+        _lib.ring_attn_set_schedule(_lib.RA_SCHEDULE_AUTO)
 
 
 def test_bounded_wait_reports_timeout_and_recovers(ra):
