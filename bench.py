@@ -136,6 +136,24 @@ def recorded_traffic(workload_name: str):
     return int(m_b.group(1))
 
 
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Largest of the ranks' device-timed milliseconds (every rank calls it,
+    in the same order)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(world: int, steps: int, flops_per_step: float, ms_max: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own copy of the workload (weak
+    scaling), so the job does world * steps forward passes in ms_max."""
+    return world * steps * flops_per_step / (ms_max / 1e3) / 1e12
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -173,7 +191,7 @@ def run_reference(args, w, world, rank):
     total_flops = total_t = 0.0
     rows = 0
     threads = os.cpu_count()
-    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    budget = getattr(args, "ref_budget", None) or max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
         fl, t, n, threads = cpu_oracle_sample(w, budget, seed=1000 + i)
         if i >= args.warmup:
@@ -245,13 +263,10 @@ def run_ours(args, w, world, rank, local):
     api.check_status(stream)
     per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     elapsed = ev[0].elapsed_time(ev[-1])
-    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_max = float(t.item())
+    elapsed_max = max_over_ranks(elapsed, world, dev)
 
     flops = w.flops()
-    value = world * args.steps * flops / (elapsed_max / 1e3) / 1e12
+    value = aggregate_throughput(world, args.steps, flops, elapsed_max)
 
     # end to end: pinned host inputs -> device, forward, outputs -> pinned host
     q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
@@ -278,10 +293,8 @@ def run_ours(args, w, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     api.check_status(stream)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * e2e_steps * flops / (float(te.item()) / 1e3) / 1e12
+    te_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = aggregate_throughput(world, e2e_steps, flops, te_max)
     h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
     d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
 
@@ -367,6 +380,8 @@ def main():
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=None,
+                    help="seconds of oracle time per reference step (default: fits the run in ~2 min)")
     args = ap.parse_args()
     from ring_attention_ordered_b200.inputs import HEADLINE, WORKLOADS
     w = WORKLOADS[args.workload or HEADLINE]
