@@ -268,7 +268,6 @@ __device__ void loader_role(const FwdParams& p, const Bars& br, uint32_t smem_ba
   using C = Cfg<D>;
   constexpr int NBOX = D / BOX_COLS;
   const bool leader = (threadIdx.x & 31) == 0;
-  const uint32_t lead = leader ? 1u : 0u;
   const int G = gridDim.x, c = blockIdx.x;
   uint32_t kv_it = 0, q_uses = 0;
   bool q_pending = false;
@@ -281,18 +280,21 @@ __device__ void loader_role(const FwdParams& p, const Bars& br, uint32_t smem_ba
       // fault injection: the first query tiles are never requested
     } else {
       const int nq = x.valid1 ? 2 : 1;
-      mbar_arrive_expect_tx_if(br.q_full, nq * C::Q_BYTES, lead);
       const int row0 = x.b * p.L + x.blk * p.blk_len;
-#pragma unroll
-      for (int bx = 0; bx < NBOX; ++bx)
-        tma_load_3d_if(smem_base + C::OFF_Q + bx * BOX_BYTES, &p.tm_q, br.q_full, bx * BOX_COLS,
-                       x.h[0], row0 + x.qt[0] * BM, lead);
-      if (x.valid1) {
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.q_full, nq * C::Q_BYTES);
 #pragma unroll
         for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d_if(smem_base + C::OFF_Q + C::Q_BYTES + bx * BOX_BYTES, &p.tm_q, br.q_full,
-                         bx * BOX_COLS, x.h[1], row0 + x.qt[1] * BM, lead);
+          tma_load_3d(smem_base + C::OFF_Q + bx * BOX_BYTES, &p.tm_q, br.q_full, bx * BOX_COLS,
+                      x.h[0], row0 + x.qt[0] * BM);
+        if (x.valid1) {
+#pragma unroll
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem_base + C::OFF_Q + C::Q_BYTES + bx * BOX_BYTES, &p.tm_q, br.q_full,
+                        bx * BOX_COLS, x.h[1], row0 + x.qt[1] * BM);
+        }
       }
+      __syncwarp();
       q_pending = true;
     }
     ++q_uses;
@@ -305,12 +307,15 @@ __device__ void loader_role(const FwdParams& p, const Bars& br, uint32_t smem_ba
         const int s = kv_it % C::NS;
         const uint32_t ph = (kv_it / C::NS) & 1u;
         if (!wait_warp(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
-        mbar_arrive_expect_tx_if(br.kv_full(s), C::KV_BYTES, lead);
         const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(br.kv_full(s), C::KV_BYTES);
 #pragma unroll
-        for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d_if(smem_base + C::OFF_KV + s * C::KV_BYTES + bx * BOX_BYTES, map,
-                         br.kv_full(s), bx * BOX_COLS, x.kvh, row, lead);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem_base + C::OFF_KV + s * C::KV_BYTES + bx * BOX_BYTES, map,
+                        br.kv_full(s), bx * BOX_COLS, x.kvh, row);
+        }
+        __syncwarp();
         ++kv_it;
       }
     }
@@ -335,19 +340,20 @@ struct QkStep {
   static constexpr uint32_t OFF = ((KK / 4) * BOX_BYTES + (KK % 4) * 32) >> 4;
 };
 
-// S = Q K^T over the head dimension: D/16 MMAs of K = 16.
+// S = Q K^T over the head dimension: D/16 MMAs of K = 16, each issued by
+// the elected lane.
 template <int D>
 __device__ __forceinline__ void mma_qk_steps(uint32_t d, uint32_t a, uint32_t b, uint32_t hi,
-                                             uint32_t idesc, uint32_t lead) {
-  mma_ss<QkStep<0>::OFF, QkStep<0>::OFF>(d, a, hi, b, hi, idesc, 0u, lead);
-  mma_ss<QkStep<1>::OFF, QkStep<1>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
-  mma_ss<QkStep<2>::OFF, QkStep<2>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
-  mma_ss<QkStep<3>::OFF, QkStep<3>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+                                             uint32_t idesc) {
+  if (elect_one()) mma_ss<QkStep<0>::OFF, QkStep<0>::OFF>(d, a, hi, b, hi, idesc, 0u);
+  if (elect_one()) mma_ss<QkStep<1>::OFF, QkStep<1>::OFF>(d, a, hi, b, hi, idesc, 1u);
+  if (elect_one()) mma_ss<QkStep<2>::OFF, QkStep<2>::OFF>(d, a, hi, b, hi, idesc, 1u);
+  if (elect_one()) mma_ss<QkStep<3>::OFF, QkStep<3>::OFF>(d, a, hi, b, hi, idesc, 1u);
   if constexpr (D == 128) {
-    mma_ss<QkStep<4>::OFF, QkStep<4>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
-    mma_ss<QkStep<5>::OFF, QkStep<5>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
-    mma_ss<QkStep<6>::OFF, QkStep<6>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
-    mma_ss<QkStep<7>::OFF, QkStep<7>::OFF>(d, a, hi, b, hi, idesc, 1u, lead);
+    if (elect_one()) mma_ss<QkStep<4>::OFF, QkStep<4>::OFF>(d, a, hi, b, hi, idesc, 1u);
+    if (elect_one()) mma_ss<QkStep<5>::OFF, QkStep<5>::OFF>(d, a, hi, b, hi, idesc, 1u);
+    if (elect_one()) mma_ss<QkStep<6>::OFF, QkStep<6>::OFF>(d, a, hi, b, hi, idesc, 1u);
+    if (elect_one()) mma_ss<QkStep<7>::OFF, QkStep<7>::OFF>(d, a, hi, b, hi, idesc, 1u);
   }
 }
 
@@ -357,12 +363,12 @@ __device__ __forceinline__ void mma_qk_steps(uint32_t d, uint32_t a, uint32_t b,
 // first MMA of the first half only.
 template <int HALF>
 __device__ __forceinline__ void mma_pv_half(uint32_t d, uint32_t p_tmem, uint32_t b, uint32_t hi,
-                                            uint32_t idesc, uint32_t acc, uint32_t lead) {
+                                            uint32_t idesc, uint32_t acc) {
   constexpr uint32_t C0 = 32 * HALF, B0 = 512 * HALF;
-  mma_ts<C0 + 0, B0 + 0>(d, p_tmem, b, hi, idesc, HALF ? 1u : acc, lead);
-  mma_ts<C0 + 8, B0 + 128>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<C0 + 16, B0 + 256>(d, p_tmem, b, hi, idesc, 1u, lead);
-  mma_ts<C0 + 24, B0 + 384>(d, p_tmem, b, hi, idesc, 1u, lead);
+  if (elect_one()) mma_ts<C0 + 0, B0 + 0>(d, p_tmem, b, hi, idesc, HALF ? 1u : acc);
+  if (elect_one()) mma_ts<C0 + 8, B0 + 128>(d, p_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<C0 + 16, B0 + 256>(d, p_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<C0 + 24, B0 + 384>(d, p_tmem, b, hi, idesc, 1u);
 }
 
 template <int D>
@@ -387,23 +393,24 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
   const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dkv0);
   const uint32_t v_lo = static_cast<uint32_t>(dv0);
   const uint32_t k_hi = static_cast<uint32_t>(dkv0 >> 32), v_hi = static_cast<uint32_t>(dv0 >> 32);
-  const uint32_t lead = leader ? 1u : 0u;
   auto issue_qk = [&](int w, int stage) {
     const uint32_t a = q_lo + ((w * C::Q_BYTES) >> 4);
     const uint32_t b = k_lo + ((stage * C::KV_BYTES) >> 4);
     const uint32_t d = tmem + w * 128;
     // k-steps of 16 elements: 32 bytes apart inside a 64-column swizzle
     // box, the next box BOX_BYTES further on
-    mma_qk_steps<D>(d, a, b, k_hi, IDESC_QK, lead);
+    mma_qk_steps<D>(d, a, b, k_hi, IDESC_QK);
   };
   auto issue_pv_half = [&](int w, int stage, int half, bool acc) {
     const uint32_t b = v_lo + ((stage * C::KV_BYTES) >> 4);
     if (half == 0)
-      mma_pv_half<0>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u, lead);
+      mma_pv_half<0>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u);
     else
-      mma_pv_half<1>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, 1u, lead);
+      mma_pv_half<1>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, 1u);
   };
-  auto commit = [&](uint32_t bar) { tc_commit_if(bar, lead); };
+  auto commit = [&](uint32_t bar) {
+    if (elect_one()) tc_commit(bar);
+  };
 
   for (int k = 0;; ++k) {
     const int u = unit_for_round(k, G, c);
@@ -427,14 +434,19 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
       ++kv_it;
       if (n == 1) commit(br.q_empty);
     }
+    // Barrier states probed ahead of time: a probe issued before a batch of
+    // MMAs overlaps its latency with their issue, and a barrier found
+    // complete is not waited on again.
+    bool rdy_v = false, rdy_k = false, rdy_p0 = false;
     for (int idx = 0; idx < n; ++idx) {
       const bool more = idx + 1 < n;
       const int vs = kv_it % C::NS;
       const int ks = (kv_it + 1) % C::NS;
-      if (!wait_warp(br.kv_full(vs), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+      if (!rdy_v && !wait_warp(br.kv_full(vs), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
       // the next K tile is needed right after P0 V: wait for it now, off the
       // softmax -> MMA -> softmax chain
-      if (more && !wait_warp(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL))
+      if (more && !rdy_k &&
+          !wait_warp(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL))
         goto drain;
       tc_fence_after();
       // query tile 0: P0 V in two halves as P0 arrives, then S0 for the next
@@ -442,7 +454,7 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
       if (idx == 0 && units0 > 0) {
         if (!wait_warp(br.o_free(0), (units0 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
       }
-      if (!wait_warp(br.p_half(0), pf_phase0, cx, SITE_P_HALF)) goto drain;
+      if (!rdy_p0 && !wait_warp(br.p_half(0), pf_phase0, cx, SITE_P_HALF)) goto drain;
       tc_fence_after();
       issue_pv_half(0, vs, 0, idx > 0);
       if (!wait_warp(br.p_full(0), pf_phase0, cx, SITE_P_FULL)) goto drain;
@@ -450,16 +462,20 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
       tc_fence_after();
       issue_pv_half(0, vs, 1, true);
       if (!more) commit(br.o_done(0));
+      // probe P1's first half now; the vote on the result comes after the
+      // S0 MMAs, so the probe's latency overlaps their issue
+      const bool raw_p1 = x.valid1 ? mbar_test_wait(br.p_half(1), pf_phase1) : true;
       if (more) {
         issue_qk(0, ks);
         commit(br.s_full(0));
       }
+      const bool rdy_p1 = __all_sync(0xffffffffu, raw_p1);
       // query tile 1
       if (x.valid1) {
         if (idx == 0 && units1 > 0) {
           if (!wait_warp(br.o_free(1), (units1 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
         }
-        if (!wait_warp(br.p_half(1), pf_phase1, cx, SITE_P_HALF)) goto drain;
+        if (!rdy_p1 && !wait_warp(br.p_half(1), pf_phase1, cx, SITE_P_HALF)) goto drain;
         tc_fence_after();
         issue_pv_half(1, vs, 0, idx > 0);
         if (!wait_warp(br.p_full(1), pf_phase1, cx, SITE_P_FULL)) goto drain;
@@ -467,13 +483,25 @@ __device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base,
         tc_fence_after();
         issue_pv_half(1, vs, 1, true);
         if (!more) commit(br.o_done(1));
-        if (more) {
+      }
+      // V of this step has been read by every P V issued so far
+      commit(br.kv_empty(vs));
+      if (more) {
+        // probe what the next step needs, then issue S1 for it
+        const bool raw_v =
+            mbar_test_wait(br.kv_full((kv_it + 2) % C::NS), ((kv_it + 2) / C::NS) & 1u);
+        const bool raw_k =
+            idx + 2 < n
+                ? mbar_test_wait(br.kv_full((kv_it + 3) % C::NS), ((kv_it + 3) / C::NS) & 1u)
+                : true;
+        const bool raw_p0 = mbar_test_wait(br.p_half(0), pf_phase0);
+        if (x.valid1) {
           issue_qk(1, ks);
           commit(br.s_full(1));
         }
-      }
-      commit(br.kv_empty(vs));
-      if (more) {
+        rdy_v = __all_sync(0xffffffffu, raw_v);
+        rdy_k = __all_sync(0xffffffffu, raw_k);
+        rdy_p0 = __all_sync(0xffffffffu, raw_p0);
         commit(br.kv_empty(ks));
         if (idx + 1 == n - 1) commit(br.q_empty);
       }
