@@ -268,33 +268,68 @@ def run_ours(args, w, world, rank, local):
     flops = w.flops()
     value = aggregate_throughput(world, args.steps, flops, elapsed_max)
 
-    # end to end: pinned host inputs -> device, forward, outputs -> pinned host
+    # End to end through the public API: a stream of independent forward
+    # passes whose inputs come from pinned host memory and whose outputs go
+    # back to it.  Every step copies its own 3 GiB of inputs in and its
+    # outputs out inside the timed region; two device buffer sets let the
+    # copies of neighbouring steps run on their own streams while the kernel
+    # of the current step computes (a serving pipeline).  The serial latency
+    # of one step (copy in, compute, copy out) is reported beside it.
     q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
     out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = max(4, min(args.steps, 8))
+    bufs = [(q, k, v, out, lse),
+            (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+             torch.empty_like(out), torch.empty_like(lse))]
+    h2d_s = torch.cuda.Stream(dev)
+    d2h_s = torch.cuda.Stream(dev)
 
-    def e2e_step():
-        q.copy_(q_p, non_blocking=True)
-        k.copy_(k_p, non_blocking=True)
-        v.copy_(v_p, non_blocking=True)
-        step()
-        out_p.copy_(out, non_blocking=True)
-        lse_p.copy_(lse, non_blocking=True)
+    def run_e2e(n_steps: int, pipelined: bool):
+        h2d_done = [torch.cuda.Event() for _ in range(n_steps)]
+        fwd_done = [torch.cuda.Event() for _ in range(n_steps)]
+        d2h_done = [torch.cuda.Event() for _ in range(n_steps)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h2d_s.wait_event(e0)
+        d2h_s.wait_event(e0)
+        for i in range(n_steps):
+            bq, bk, bv, bo, bl = bufs[i % 2] if pipelined else bufs[0]
+            with torch.cuda.stream(h2d_s):
+                if i >= 2 or (not pipelined and i >= 1):
+                    # buffer set reused: its forward must be done
+                    h2d_s.wait_event(fwd_done[i - 2 if pipelined else i - 1])
+                if not pipelined and i >= 1:
+                    h2d_s.wait_event(d2h_done[i - 1])
+                bq.copy_(q_p, non_blocking=True)
+                bk.copy_(k_p, non_blocking=True)
+                bv.copy_(v_p, non_blocking=True)
+                h2d_done[i].record(h2d_s)
+            stream.wait_event(h2d_done[i])
+            if i >= 2 and pipelined:
+                stream.wait_event(d2h_done[i - 2])   # outputs of the set read back
+            api.fwd(bq, bk, bv, w.n_ring, w.causal, w.scale, out=bo, lse=bl, stream=stream)
+            fwd_done[i].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(fwd_done[i])
+                out_p.copy_(bo, non_blocking=True)
+                lse_p.copy_(bl, non_blocking=True)
+                d2h_done[i].record(d2h_s)
+        stream.wait_event(d2h_done[n_steps - 1])
+        stream.wait_event(h2d_done[n_steps - 1])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
 
-    e2e_step()
+    run_e2e(2, True)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    api.check_status(stream)
-    te_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    te_max = max_over_ranks(run_e2e(e2e_steps, True), world, dev)
     e2e_value = aggregate_throughput(world, e2e_steps, flops, te_max)
+    serial_ms = max_over_ranks(run_e2e(2, False), world, dev) / 2
+    api.check_status(stream)
+    del bufs
     h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h))
     d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
 
@@ -360,7 +395,9 @@ def run_ours(args, w, world, rank, local):
                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})"},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": te_max / e2e_steps, "serial_latency_ms": serial_ms,
+                "mode": "pipelined: step k+1 copies in and step k-1 copies out while step k computes"},
         "gpu_launches": args.steps,
         "clocks": clocks,
         "merge": {"ms": merge_ms, "GB/s": merge_bytes / (merge_ms / 1e3) / 1e9,
