@@ -408,6 +408,53 @@ def run_ours(args, w, world, rank, local):
     return 0
 
 
+def run_all_workloads(args):
+    """Per-workload forward throughput on one GPU (not the contract line):
+    one JSON line per workload with ms, TFLOP/s, tokens/s and the fractions of
+    the measured bf16 peaks, plus the SM clock seen during its timed region."""
+    import torch
+
+    from ring_attention_ordered_b200 import _lib, api
+    from ring_attention_ordered_b200.inputs import WORKLOADS, workload_inputs
+
+    _lib.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    for name, w in WORKLOADS.items():
+        q_h, k_h, v_h = workload_inputs(w)
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        del q_h, k_h, v_h
+        out = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+        steps = 2 if w.L >= 1 << 20 else (10 if w.L >= 1 << 15 else 50)
+        for _ in range(3):
+            api.fwd(q, k, v, w.n_ring, w.causal, w.scale, out=out, lse=lse, stream=stream)
+        api.check_status(stream)
+        sampler = ClockSampler(0)
+        sampler.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            api.fwd(q, k, v, w.n_ring, w.causal, w.scale, out=out, lse=lse, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks = sampler.stop()
+        api.check_status(stream)
+        ms = e0.elapsed_time(e1) / steps
+        tflops = w.flops() / (ms / 1e3) / 1e12
+        print(json.dumps({
+            "kind": "workload", "workload": w.describe(), "name": name, "steps": steps,
+            "ms": ms, "TFLOP/s": tflops, "tokens_per_s": w.B * w.L / (ms / 1e3),
+            "frac_of_burst": tflops / peaks["bf16_tflops"],
+            "frac_of_sustained": tflops / peaks["bf16_tflops_sustained"],
+            "clocks": clocks}), flush=True)
+        del q, k, v, out, lse
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,6 +464,8 @@ def main():
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="print one line per named workload instead of the benchmark line")
     ap.add_argument("--ref-budget", type=float, default=None,
                     help="seconds of oracle time per reference step (default: fits the run in ~2 min)")
     args = ap.parse_args()
@@ -427,6 +476,8 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args, w, world, rank)
+    if args.all_workloads:
+        return run_all_workloads(args)
     return run_ours(args, w, world, rank, local)
 
 

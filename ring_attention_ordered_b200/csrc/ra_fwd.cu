@@ -67,11 +67,13 @@ constexpr float RESCALE_LOG2 = 8.0f;
 // one MUFU ex2 per score element would keep MUFU exactly as busy as the
 // tensor core, so part of the exponentials move to the otherwise idle FMA
 // pipe.
-#ifndef RA_EMU_COLS
-#define RA_EMU_COLS 0
+// Column pairs j (0..63) with (j % EMU_PERIOD) == EMU_PERIOD - 1 use the
+// polynomial; 0 disables it.  Spreading them across the row lets the
+// scheduler overlap them with the MUFU work of the other pairs.
+#ifndef RA_EMU_PERIOD
+#define RA_EMU_PERIOD 0
 #endif
-constexpr int EMU_COLS = RA_EMU_COLS;
-static_assert(EMU_COLS % 2 == 0 && EMU_COLS >= 0 && EMU_COLS <= 128, "emulated columns");
+constexpr int EMU_PERIOD = RA_EMU_PERIOD;
 // Longest single hardware suspension inside one mbarrier try_wait (ns).
 #ifndef RA_WAIT_HINT_NS
 #define RA_WAIT_HINT_NS 1000000u
@@ -539,8 +541,8 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1) {
   float q0, q1, t0, t1;
   f2_unpack(q, q0, q1);
   f2_unpack(t, t0, t1);
-  r0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  r1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+  r0 = __uint_as_float(__float_as_uint(q0) + __float_as_uint(t0) * 8388608u);
+  r1 = __uint_as_float(__float_as_uint(q1) + __float_as_uint(t1) * 8388608u);
 }
 
 // One score row (128 columns held in sr): P = 2^(s * c2 - m) written as bf16
@@ -566,7 +568,7 @@ __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, fl
       const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])),
                                  c2x2, nm2);
       float p0, p1;
-      if (col < EMU_COLS) {
+      if (EMU_PERIOD > 0 && (j % (EMU_PERIOD > 0 ? EMU_PERIOD : 1)) == EMU_PERIOD - 1) {
         exp2_poly2(x2, p0, p1);
       } else {
         float x0, x1;
