@@ -26,6 +26,7 @@ from .attn_fp64 import (  # noqa: F401
     attention,
     attention_rows,
     attention_probs,
+    block_attention,
     brute_attention,
     ring_order,
     ring_visits,

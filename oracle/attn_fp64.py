@@ -210,6 +210,52 @@ def _block_scores(qi, kj, scale, kind):
     return s
 
 
+def block_attention(q, k, v, scale: float, kind: str):
+    """Exact attention of one query block against one K/V block, as a partial
+    result (o, lse) over the keys the visit allows -- what one host computes on
+    one ring step before folding it into its output ("Ring Attention 环注意力",
+    L4 §4.2 steps 1-2).  Local rows r of the query block, c of the K/V block:
+
+    * ``"full"``: every key (an earlier block, or no causal mask);
+    * ``"masked"``: keys c <= r (the host's own block under causal masking);
+    * ``"strict"``: keys c < r (a striped layout's block from a later host,
+      "Striped Attention" in L4 §4.8: its key at local row r comes after the
+      query in the sequence).
+
+    A row with no allowed key is the empty partial: o = 0, lse = -inf.
+    q [B, lq, Hq, d], k/v [B, lk, Hkv, d] (lq == lk unless ``"full"``).
+    Returns o [B, lq, Hq, d], lse [B, Hq, lq] in float64.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, lq, Hq, d = q.shape
+    _, lk, Hkv, _ = k.shape
+    if kind not in ("full", "masked", "strict"):
+        raise ValueError(f"unknown visit kind {kind!r}")
+    if kind != "full" and lq != lk:
+        raise ValueError("masked visits need equal block lengths")
+    g = Hq // Hkv
+    o = np.zeros((B, lq, Hq, d))
+    lse = np.full((B, Hq, lq), NEG_INF)
+    rows = np.arange(lq)[:, None]
+    cols = np.arange(lk)[None, :]
+    allowed = np.ones((lq, lk), dtype=bool)
+    if kind == "masked":
+        allowed = cols <= rows
+    elif kind == "strict":
+        allowed = cols < rows
+    live = allowed.any(axis=1)
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * (q[b, :, h, :] @ k[b, :, h // g, :].T)
+            s = np.where(allowed, s, NEG_INF)[live]
+            if s.shape[0] == 0:
+                continue
+            o_r, l_r = _softmax_weighted_sum(s, v[b, :, h // g, :])
+            o[b, live, h, :] = o_r
+            lse[b, h, live] = l_r
+    return o, lse
+
+
 def ring_attention(q, k, v, n_ring: int, causal: bool, scale: float):
     """Ring attention emulated on one host, with the running accumulator.
 

@@ -465,3 +465,90 @@ def test_planted_merge_mistake_is_caught(mistake):
         lse = np.log(den) if mistake == "no_max_shift_in_lse" else mx + np.log(den)
         return o, lse
     assert _fails(pin_merge_split_keys, mutant, oracle.attention) or _fails(pin_merge_closed_forms, mutant)
+
+
+# --------------------------------------------------------------------------
+# block_attention: one ring visit as a partial result
+# --------------------------------------------------------------------------
+
+def pin_block_full_and_masked(block):
+    """"full" and "masked" visits are plain and causal attention of the
+    block, checked against the exactly rounded brute force."""
+    rng = np.random.default_rng(21)
+    q, k, v = rand(2, 7, 4, 5, rng=rng), rand(2, 7, 2, 5, rng=rng), rand(2, 7, 2, 5, rng=rng)
+    for kind, causal in (("full", False), ("masked", True)):
+        o, l_ = block(q, k, v, 0.6, kind)
+        ob, lb = oa.brute_attention(q, k, v, causal, 0.6)
+        np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l_, lb, rtol=0, atol=1e-12)
+
+
+def pin_block_strict_is_shifted_causal(block):
+    """"strict" (keys c < r): row r of the block sees keys 0..r-1, which is
+    row r-1 of causal attention of q[1:] against k[:-1], v[:-1] (brute
+    force); row 0 has no key: o = 0, lse = -inf."""
+    rng = np.random.default_rng(22)
+    q, k, v = rand(1, 8, 2, 4, rng=rng), rand(1, 8, 1, 4, rng=rng), rand(1, 8, 1, 4, rng=rng)
+    o, l_ = block(q, k, v, 0.8, "strict")
+    ob, lb = oa.brute_attention(q[:, 1:], k[:, :-1], v[:, :-1], True, 0.8)
+    np.testing.assert_allclose(o[:, 1:], ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l_[:, :, 1:], lb, rtol=0, atol=1e-12)
+    assert np.all(o[:, 0] == 0.0) and np.all(l_[:, :, 0] == -np.inf)
+
+
+def pin_block_unequal_lengths(block):
+    """A "full" visit of 5 query rows against 11 keys: torch's fp64
+    scaled_dot_product_attention (a library routine) with GQA grouping."""
+    rng = np.random.default_rng(23)
+    q, k, v = rand(1, 5, 4, 8, rng=rng), rand(1, 11, 2, 8, rng=rng), rand(1, 11, 2, 8, rng=rng)
+    o, _ = block(q, k, v, 0.35, "full")
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.35,
+                                                           enable_gqa=True)
+    np.testing.assert_allclose(o, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+
+
+BLOCK_PINS = [pin_block_full_and_masked, pin_block_strict_is_shifted_causal,
+              pin_block_unequal_lengths]
+
+
+@pytest.mark.parametrize("pin", BLOCK_PINS)
+def test_block_attention_pins(pin):
+    pin(oracle.block_attention)
+
+
+def _mutant_block(mistake):
+    def block(q, k, v, scale, kind):
+        q, k, v = oa._f64(q), oa._f64(k), oa._f64(v)
+        B, lq, Hq, d = q.shape
+        lk, Hkv = k.shape[1], k.shape[2]
+        o = np.zeros((B, lq, Hq, d))
+        lse = np.full((B, Hq, lq), -np.inf)
+        r, c = np.arange(lq)[:, None], np.arange(lk)[None, :]
+        allowed = np.ones((lq, lk), bool)
+        if kind == "masked":
+            allowed = c <= r
+        elif kind == "strict":
+            allowed = (c <= r) if mistake == "strict_keeps_diagonal" else (c < r)
+        for b in range(B):
+            for h in range(Hq):
+                s = scale * (q[b, :, h] @ k[b, :, h // (Hq // Hkv)].T)
+                s = np.where(allowed, s, -np.inf)
+                for i in range(lq):
+                    if not allowed[i].any():
+                        if mistake == "empty_row_uniform":
+                            o[b, i, h] = v[b, :, h // (Hq // Hkv)].mean(axis=0)
+                        continue
+                    m = s[i].max()
+                    e = np.exp(s[i] - m)
+                    o[b, i, h] = e @ v[b, :, h // (Hq // Hkv)] / e.sum()
+                    lse[b, h, i] = m + np.log(e.sum()) + (1.0 if mistake == "lse_plus_one" else 0.0)
+        return o, lse
+    return block
+
+
+@pytest.mark.parametrize("mistake", ["strict_keeps_diagonal", "empty_row_uniform", "lse_plus_one"])
+def test_planted_block_mistake_is_caught(mistake):
+    assert any(_fails(pin, _mutant_block(mistake)) for pin in BLOCK_PINS), mistake
+    for pin in BLOCK_PINS:
+        pin(_mutant_block(None))
