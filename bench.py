@@ -455,6 +455,74 @@ def run_all_workloads(args):
     return 0
 
 
+def run_ring_emulated(args, w):
+    """The multi-host ring's compute, host by host, on one GPU (not the
+    contract line).  For each layout, every host's visit sequence on the
+    workload (its n_ring hosts) is timed alone with CUDA events, as that host
+    would run it on its own GPU; the exchange is not part of it.  The ring's
+    compute time is the slowest host's; one JSON line per layout gives the
+    per-host times, that critical path, the throughput it implies for the
+    n_ring-GPU job and its ratio to n_ring times the fused single-GPU kernel."""
+    import torch
+
+    from ring_attention_ordered_b200 import _lib, api, ring
+    from ring_attention_ordered_b200.inputs import workload_inputs
+
+    _lib.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    q_h, k_h, v_h = workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    del q_h, k_h, v_h
+    N = w.n_ring
+    steps = max(1, args.steps)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        api.check_status(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        api.check_status(stream)
+        return e0.elapsed_time(e1) / steps
+
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    fused_ms = timed(lambda: api.fwd(q, k, v, N, w.causal, w.scale, out=out, lse=lse,
+                                     stream=stream))
+    del out, lse
+    for layout in ring.LAYOUTS:
+        ks = [ring.shard(k, h, N, layout) for h in range(N)]
+        vs = [ring.shard(v, h, N, layout) for h in range(N)]
+        host_ms, host_launches = [], []
+        for host in range(N):
+            qh = ring.shard(q, host, N, layout)
+            plan = ring.visit_plan(host, N, w.causal, layout)
+            host_launches.append(sum(len(vs_) for _, vs_ in plan))
+            host_ms.append(timed(lambda: ring._run_host(
+                qh, lambda t: ks[plan[t][0]], lambda t: vs[plan[t][0]], plan, w.scale,
+                ring.cuda_visit)))
+            del qh
+        crit = max(host_ms)
+        tflops = w.flops() / (crit / 1e3) / 1e12
+        print(json.dumps({
+            "kind": "ring_emulated", "workload": w.describe(), "layout": layout, "hosts": N,
+            "host_ms": host_ms, "host_launches": host_launches, "critical_ms": crit,
+            "sum_ms": sum(host_ms), "job_TFLOP/s_compute_only": tflops,
+            "per_gpu_frac_of_burst": tflops / N / peaks["bf16_tflops"],
+            "fused_1gpu_ms": fused_ms,
+            "frac_of_fused_over_N": fused_ms / (N * crit)}), flush=True)
+        del ks, vs
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,6 +534,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--all-workloads", action="store_true",
                     help="print one line per named workload instead of the benchmark line")
+    ap.add_argument("--ring-emulated", action="store_true",
+                    help="time every host of the multi-host ring on this GPU (three layouts)")
     ap.add_argument("--ref-budget", type=float, default=None,
                     help="seconds of oracle time per reference step (default: fits the run in ~2 min)")
     args = ap.parse_args()
@@ -478,6 +548,8 @@ def main():
         return run_reference(args, w, world, rank)
     if args.all_workloads:
         return run_all_workloads(args)
+    if args.ring_emulated:
+        return run_ring_emulated(args, w)
     return run_ours(args, w, world, rank, local)
 
 

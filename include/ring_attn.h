@@ -79,6 +79,51 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                         float scale, ra_stream_t stream);
 
 /*
+ * ring_attn_fwd_visit -- one ring step of one host: its query block against
+ * the K/V block it holds at that step, folded into its running output
+ * ("Ring Attention 环注意力" L4 §4.2 steps 1-2: compute on the block in
+ * hand, accumulate into O_i, pass K/V on; the striped and zigzag layouts of
+ * L4 §4.5 limitation 2 and §4.8 use the same visits on other row sets).
+ * A multi-device ring calls this once per step while the next K/V block is
+ * in flight; the exchange itself is the caller's (the Python ring driver
+ * uses torch.distributed send/recv).
+ *
+ * For every batch b, query head h and row r of the block (l rows):
+ *     o_t[b, r, h, :] = sum_c softmax_c(scale * q[b,r,h,:] . k[b,c,h/g,:]) v[b,c,h/g,:]
+ *     lse_t[b, h, r]  = ln sum_c exp(scale * q[b,r,h,:] . k[b,c,h/g,:])
+ * over the keys c of the K/V block allowed by `diag`:
+ *   diag == 0: all c (a block earlier in the sequence, or no causal mask);
+ *   diag == 1: c <= r (the host's own block under causal masking, or, in a
+ *              striped layout, a block from a host at or before this one);
+ *   diag == 2: c < r (striped layout, a block from a later host: its key at
+ *              local row r follows the query in the sequence).  Local row 0
+ *              has no key: its partial is empty, o_t = 0 and lse_t = -inf,
+ *              which the fold ignores (on the first visit o_acc row = 0,
+ *              lse_acc = -inf).
+ * fold == 0: o_acc = o_t, lse_acc = lse_t (the first visit).
+ * fold == 1: (o_acc, lse_acc) = merge((o_acc, lse_acc), (o_t, lse_t)) with
+ *   the row merge of ring_attn_merge, bitwise the same as writing o_t/lse_t
+ *   to separate buffers and merging them with ring_attn_merge.
+ * out, if not NULL, receives the bf16 (round to nearest even) copy of the
+ * new o_acc: pass it on the last visit to get the finished output.
+ *
+ *   q       bf16 [B, l, Hq,  d] contiguous: the host's query block     (in)
+ *   k, v    bf16 [B, l, Hkv, d] contiguous: the visited K/V block      (in)
+ *   o_acc   fp32 [B, l, Hq,  d] contiguous (read when fold == 1)    (in/out)
+ *   lse_acc fp32 [B, Hq, l] contiguous, natural log (read when fold) (in/out)
+ *   out     bf16 [B, l, Hq,  d] contiguous, or NULL                    (out)
+ *   B, Hq, Hkv, l, d   as for ring_attn_fwd with L = l, n_ring = 1.
+ *   diag 0, 1 or 2; fold 0 or 1; scale finite and >= 0.
+ *
+ * Pointers must be 16-byte aligned; o_acc, lse_acc and out must not overlap
+ * the inputs or each other.  B*Hq*l == 0 launches nothing.  Errors as for
+ * ring_attn_fwd; nothing is written on an argument error.
+ */
+ra_status ring_attn_fwd_visit(const void* q, const void* k, const void* v, float* o_acc,
+                              float* lse_acc, void* out, int B, int Hq, int Hkv, int64_t l, int d,
+                              int diag, int fold, float scale, ra_stream_t stream);
+
+/*
  * ring_attn_merge -- fold two partial attention results over disjoint key
  * sets into one (the accumulation of each ring step's blockwise result into
  * O_i, "Ring Attention 环注意力" L4 §4.2 step 2, kept as output plus

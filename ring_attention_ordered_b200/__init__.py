@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     ring_attn_check_status,
     ring_attn_debug_inject,
     ring_attn_fwd,
+    ring_attn_fwd_visit,
     ring_attn_merge,
     ring_attn_set_max_ctas,
     ring_attn_set_schedule,

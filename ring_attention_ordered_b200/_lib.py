@@ -23,6 +23,8 @@ _I = ctypes.c_int
 _I64 = ctypes.c_int64
 SIGNATURES = {
     "ring_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, ctypes.c_float, _P]),
+    "ring_attn_fwd_visit": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I,
+                                 ctypes.c_float, _P]),
     "ring_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I, _P]),
     "ring_attn_check_status": (_I, [_P]),
     "ring_attn_set_wait_limit_ns": (_I, [ctypes.c_uint64]),
@@ -77,6 +79,12 @@ def _check(status: int) -> int:
 def ring_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, L, d, n_ring, causal, scale, stream=0):
     return _check(load().ring_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, L, d, n_ring,
                                        int(bool(causal)), float(scale), stream))
+
+
+def ring_attn_fwd_visit(q, k, v, o_acc, lse_acc, out, B, Hq, Hkv, l, d, diag, fold, scale,
+                        stream=0):
+    return _check(load().ring_attn_fwd_visit(q, k, v, o_acc, lse_acc, out, B, Hq, Hkv, l, d,
+                                             int(diag), int(fold), float(scale), stream))
 
 
 def ring_attn_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d, stream=0):

@@ -52,6 +52,38 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: 
     return out, lse
 
 
+def fwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Tensor,
+              lse_acc: torch.Tensor, diag: int, fold: bool, scale: float | None = None,
+              out: torch.Tensor | None = None, stream=None):
+    """One ring visit: the query block q [B, l, Hq, d] against the K/V block
+    k/v [B, l, Hkv, d] (bf16), written to (fold=False) or folded into
+    (fold=True) the running fp32 accumulator o_acc [B, l, Hq, d] and
+    lse_acc [B, Hq, l].  ``diag``: 0 every key, 1 keys c <= r, 2 keys c < r
+    (local rows).  ``out`` (bf16, optional) receives the rounded
+    accumulator.  Returns (o_acc, lse_acc, out)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_cuda(t, n, torch.bfloat16, 4)
+    B, l, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, l, Hkv, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
+    _check_cuda(o_acc, "o_acc", torch.float32, 4)
+    _check_cuda(lse_acc, "lse_acc", torch.float32, 3)
+    if o_acc.shape != q.shape or lse_acc.shape != (B, Hq, l):
+        raise ValueError("o_acc/lse_acc shapes do not match q")
+    if out is not None:
+        _check_cuda(out, "out", torch.bfloat16, 4)
+        if out.shape != q.shape:
+            raise ValueError("out shape does not match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(q.device):
+        _lib.ring_attn_fwd_visit(q.data_ptr(), k.data_ptr(), v.data_ptr(), o_acc.data_ptr(),
+                                 lse_acc.data_ptr(), 0 if out is None else out.data_ptr(),
+                                 B, Hq, Hkv, l, d, diag, fold, scale, _stream_handle(stream))
+    return o_acc, lse_acc, out
+
+
 def merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,
           out: torch.Tensor | None = None, lse_out: torch.Tensor | None = None, stream=None):
     """Log-sum-exp merge of two partials: o [rows, d] fp32, lse [rows] fp32."""

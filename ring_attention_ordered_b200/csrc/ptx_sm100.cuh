@@ -111,6 +111,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_if(uint32_t bar, uint32_t 
       :: "r"(bar), "r"(bytes), "r"(issue) : "memory");
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" :: "l"(reinterpret_cast<uint64_t>(p)));
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -110,41 +110,11 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-}  // namespace
-
-extern "C" {
-
-ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
-                        int Hq, int Hkv, int64_t L, int d, int n_ring, int causal, float scale,
-                        ra_stream_t stream) {
-  if (B < 0 || Hq < 0 || Hkv < 0 || L < 0)
-    return fail(RA_ERR_INVALID_ARG, "negative size (B=%d Hq=%d Hkv=%d L=%lld)", B, Hq, Hkv,
-                static_cast<long long>(L));
-  if (n_ring < 1) return fail(RA_ERR_INVALID_ARG, "n_ring must be >= 1 (got %d)", n_ring);
-  if (causal != 0 && causal != 1) return fail(RA_ERR_INVALID_ARG, "causal must be 0 or 1");
-  if (!std::isfinite(scale) || scale < 0.f)
-    return fail(RA_ERR_INVALID_ARG, "scale must be finite and >= 0");
-  if (L % n_ring != 0)
-    return fail(RA_ERR_INVALID_ARG, "L=%lld does not split into %d equal blocks",
-                static_cast<long long>(L), n_ring);
-  if (Hkv == 0 && Hq != 0) return fail(RA_ERR_INVALID_ARG, "Hkv must be >= 1");
-  if (Hkv > 0 && Hq % Hkv != 0)
-    return fail(RA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
-  if (d != 64 && d != 128) return fail(RA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-  if (static_cast<long long>(B) * Hq * L == 0) return ok();
-  if (static_cast<long long>(B) * L >= (1ll << 31))
-    return fail(RA_ERR_INVALID_ARG, "B*L must be < 2^31");
-  if (!q || !k || !v || !out || !lse) return fail(RA_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
-    return fail(RA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  const size_t nq = static_cast<size_t>(B) * L * Hq * d * 2;
-  const size_t nkv = static_cast<size_t>(B) * L * Hkv * d * 2;
-  const size_t nl = static_cast<size_t>(B) * Hq * L * 4;
-  if (overlaps(out, nq, q, nq) || overlaps(out, nq, k, nkv) || overlaps(out, nq, v, nkv) ||
-      overlaps(lse, nl, q, nq) || overlaps(lse, nl, k, nkv) || overlaps(lse, nl, v, nkv) ||
-      overlaps(out, nq, lse, nl))
-    return fail(RA_ERR_INVALID_ARG, "outputs overlap the inputs or each other");
-
+// Shared by ring_attn_fwd and ring_attn_fwd_visit: tensor maps, work units,
+// schedule and launch of the forward kernel.  Arguments are already checked.
+ra_status launch_forward(const void* q, const void* k, const void* v, void* out, float* lse,
+                         float* o_acc, int visit_fold, int diag_shift, int B, int Hq, int Hkv, int64_t L, int d,
+                         int n_ring, int causal, float scale, size_t nkv, ra_stream_t stream) {
   int sms = 0;
   ra_status st = device_info(&sms);
   if (st != RA_OK) return st;
@@ -157,6 +127,9 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   if ((st = make_map(&prm.tm_v, v, Hkv, rows, d)) != RA_OK) return st;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
+  prm.o_acc = o_acc;
+  prm.visit_fold = visit_fold;
+  prm.diag_shift = diag_shift;
   prm.B = B;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -189,6 +162,81 @@ ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   cudaError_t e = ra::launch_fwd(prm, d, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "forward launch: %s", cudaGetErrorString(e));
   return ok();
+}
+
+// Checks common to both forward entry points (sizes, values, head dim).
+ra_status check_forward_shape(int B, int Hq, int Hkv, int64_t L, int d, int n_ring, int causal,
+                              float scale) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || L < 0)
+    return fail(RA_ERR_INVALID_ARG, "negative size (B=%d Hq=%d Hkv=%d L=%lld)", B, Hq, Hkv,
+                static_cast<long long>(L));
+  if (n_ring < 1) return fail(RA_ERR_INVALID_ARG, "n_ring must be >= 1 (got %d)", n_ring);
+  if (causal != 0 && causal != 1) return fail(RA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (!std::isfinite(scale) || scale < 0.f)
+    return fail(RA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (L % n_ring != 0)
+    return fail(RA_ERR_INVALID_ARG, "L=%lld does not split into %d equal blocks",
+                static_cast<long long>(L), n_ring);
+  if (Hkv == 0 && Hq != 0) return fail(RA_ERR_INVALID_ARG, "Hkv must be >= 1");
+  if (Hkv > 0 && Hq % Hkv != 0)
+    return fail(RA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(RA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (static_cast<long long>(B) * Hq * L != 0 && static_cast<long long>(B) * L >= (1ll << 31))
+    return fail(RA_ERR_INVALID_ARG, "B*L must be < 2^31");
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ra_status ring_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                        int Hq, int Hkv, int64_t L, int d, int n_ring, int causal, float scale,
+                        ra_stream_t stream) {
+  ra_status st = check_forward_shape(B, Hq, Hkv, L, d, n_ring, causal, scale);
+  if (st != RA_OK) return st;
+  if (static_cast<long long>(B) * Hq * L == 0) return ok();
+  if (!q || !k || !v || !out || !lse) return fail(RA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(RA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t nq = static_cast<size_t>(B) * L * Hq * d * 2;
+  const size_t nkv = static_cast<size_t>(B) * L * Hkv * d * 2;
+  const size_t nl = static_cast<size_t>(B) * Hq * L * 4;
+  if (overlaps(out, nq, q, nq) || overlaps(out, nq, k, nkv) || overlaps(out, nq, v, nkv) ||
+      overlaps(lse, nl, q, nq) || overlaps(lse, nl, k, nkv) || overlaps(lse, nl, v, nkv) ||
+      overlaps(out, nq, lse, nl))
+    return fail(RA_ERR_INVALID_ARG, "outputs overlap the inputs or each other");
+  return launch_forward(q, k, v, out, lse, nullptr, 0, 0, B, Hq, Hkv, L, d, n_ring, causal, scale,
+                        nkv, stream);
+}
+
+ra_status ring_attn_fwd_visit(const void* q, const void* k, const void* v, float* o_acc,
+                              float* lse_acc, void* out, int B, int Hq, int Hkv, int64_t l, int d,
+                              int diag, int fold, float scale, ra_stream_t stream) {
+  if (diag < 0 || diag > 2) return fail(RA_ERR_INVALID_ARG, "diag must be 0, 1 or 2");
+  if (fold != 0 && fold != 1) return fail(RA_ERR_INVALID_ARG, "fold must be 0 or 1");
+  ra_status st = check_forward_shape(B, Hq, Hkv, l, d, 1, diag != 0, scale);
+  if (st != RA_OK) return st;
+  if (static_cast<long long>(B) * Hq * l == 0) return ok();
+  if (!q || !k || !v || !o_acc || !lse_acc) return fail(RA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_acc) || !aligned16(lse_acc) ||
+      !aligned16(out))
+    return fail(RA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t nq = static_cast<size_t>(B) * l * Hq * d * 2;
+  const size_t nkv = static_cast<size_t>(B) * l * Hkv * d * 2;
+  const size_t no = 2 * nq;
+  const size_t nl = static_cast<size_t>(B) * Hq * l * 4;
+  const void* ins[3] = {q, k, v};
+  const size_t in_n[3] = {nq, nkv, nkv};
+  for (int i = 0; i < 3; ++i)
+    if (overlaps(o_acc, no, ins[i], in_n[i]) || overlaps(lse_acc, nl, ins[i], in_n[i]) ||
+        (out && overlaps(out, nq, ins[i], in_n[i])))
+      return fail(RA_ERR_INVALID_ARG, "outputs overlap the inputs");
+  if (overlaps(o_acc, no, lse_acc, nl) || (out && (overlaps(out, nq, o_acc, no) ||
+                                                   overlaps(out, nq, lse_acc, nl))))
+    return fail(RA_ERR_INVALID_ARG, "o_acc, lse_acc and out overlap each other");
+  return launch_forward(q, k, v, out, lse_acc, o_acc, fold, diag == 2, B, Hq, Hkv, l, d, 1,
+                        diag != 0, scale, nkv, stream);
 }
 
 ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b,
@@ -271,6 +319,6 @@ const char* ring_attn_status_string(ra_status s) {
 
 const char* ring_attn_last_error(void) { return g_last_error.c_str(); }
 
-int ring_attn_version(void) { return 100; }
+int ring_attn_version(void) { return 101; }
 
 }  // extern "C"

@@ -41,6 +41,7 @@
 
 #include "ptx_sm100.cuh"
 #include "ra_internal.h"
+#include "ra_merge_math.cuh"
 #include "ring_attn.h"
 
 namespace ra {
@@ -598,6 +599,55 @@ __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, fl
   return a + b;
 }
 
+// Epilogue of a per-visit launch: this visit's normalised rows O / l (fp32)
+// are folded into the running accumulator o_acc / lse with the row merge of
+// the merge kernel (bitwise the same as writing them and merging), or
+// overwrite it on the first visit; `out` optionally gets the bf16 rounding.
+// The accumulator row was prefetched into L2 during the unit's last K/V step.
+template <int D>
+__device__ __forceinline__ void visit_epilogue(const FwdParams& p, uint32_t tO, bool row_ok, int b,
+                                               long long pos, int h, float inv_l, float lse_t) {
+  const long long row = (static_cast<long long>(b) * p.L + pos) * p.Hq + h;
+  float* lse_dst = p.lse + (static_cast<long long>(b) * p.Hq + h) * p.L + pos;
+  float4* acc = reinterpret_cast<float4*>(p.o_acc + row * D);
+  uint4* out4 = reinterpret_cast<uint4*>(p.out + row * D);
+  MergeW mw;
+  if (p.visit_fold && row_ok) mw = merge_weights(*lse_dst, lse_t);
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32(tO + cc * 32, o);
+    tmem_wait_ld();
+    float r[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r[j] = __uint_as_float(o[j]) * inv_l;
+    if (row_ok) {
+      if (p.visit_fold) {
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 a = acc[cc * 8 + c4];
+          r[4 * c4 + 0] = merge_one(mw, a.x, r[4 * c4 + 0]);
+          r[4 * c4 + 1] = merge_one(mw, a.y, r[4 * c4 + 1]);
+          r[4 * c4 + 2] = merge_one(mw, a.z, r[4 * c4 + 2]);
+          r[4 * c4 + 3] = merge_one(mw, a.w, r[4 * c4 + 3]);
+        }
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4)
+        acc[cc * 8 + c4] = make_float4(r[4 * c4], r[4 * c4 + 1], r[4 * c4 + 2], r[4 * c4 + 3]);
+      if (p.out != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          out4[cc * 4 + j] =
+              make_uint4(pack_bf16x2(r[8 * j], r[8 * j + 1]), pack_bf16x2(r[8 * j + 2], r[8 * j + 3]),
+                         pack_bf16x2(r[8 * j + 4], r[8 * j + 5]),
+                         pack_bf16x2(r[8 * j + 6], r[8 * j + 7]));
+      }
+    }
+  }
+  if (row_ok) *lse_dst = p.visit_fold ? mw.lse : lse_t;
+}
+
 template <int D>
 __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, int w,
                              const Ctl& cx) {
@@ -628,8 +678,15 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
       // tcgen05.st, which all 32 lanes must execute together; lanes whose own
       // row needs no mask (lim = 127) run the masked code harmlessly.
       int lim = min(BN, p.blk_len - it.kl * BN) - 1;
-      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * BN);
+      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * BN - p.diag_shift);
       const bool masked = __any_sync(0xffffffffu, lim < BN - 1);
+      if (p.o_acc != nullptr && p.visit_fold && idx == x.n_kv - 1 && qrow < p.blk_len) {
+        // the epilogue reads this row of the running accumulator (D fp32) back
+        const char* a = reinterpret_cast<const char*>(
+            p.o_acc + ((static_cast<long long>(x.b) * p.L + qrow) * p.Hq + h) * D);
+#pragma unroll
+        for (int c = 0; c < D * 4; c += 128) prefetch_l2(a + c);
+      }
 
       bool ok = wait_bar(br.s_full(w), s_phase, cx, SITE_S_FULL);
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -706,6 +763,15 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
       const bool row_ok = qrow < p.blk_len;
       const long long pos = static_cast<long long>(x.blk) * p.blk_len + qrow;
       const float inv_l = 1.f / l;
+      if (p.o_acc != nullptr) {
+        // a row with no allowed key (strict diagonal, row 0) is an empty
+        // partial: o = 0, lse = -inf, which the fold ignores
+        visit_epilogue<D>(p, tO, row_ok, x.b, pos, h, l > 0.f ? inv_l : 0.f, (m + log2f(l)) * LN2);
+        tc_fence_before();
+        mbar_arrive(br.o_free(w));
+        ++units_w;
+        continue;
+      }
       __nv_bfloat16* dst = p.out + ((static_cast<long long>(x.b) * p.L + pos) * p.Hq + h) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {

@@ -17,8 +17,16 @@ struct FwdParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  __nv_bfloat16* out;
+  __nv_bfloat16* out;  // bf16 output; may be NULL in a per-visit launch
   float* lse;
+  // Per-visit launch (o_acc != NULL): the whole launch is one ring visit of a
+  // query block against one K/V block (n_ring == 1, causal == diagonal
+  // visit); its fp32 result goes to o_acc [B, L, Hq, d] and lse, folded into
+  // what they hold when visit_fold == 1, and out (if not NULL) receives the
+  // bf16 rounding of the folded result.
+  float* o_acc;
+  int visit_fold;
+  int diag_shift;      // 1: the diagonal visit excludes the key at the query's own row
   int B, Hq, Hkv, group;
   int L, blk_len, n_ring, causal;
   int tiles_per_blk;   // ceil(blk_len / 128)

@@ -19,48 +19,12 @@
 #include <cstdint>
 
 #include "ra_internal.h"
+#include "ra_merge_math.cuh"
 
 namespace ra {
 
 constexpr int MERGE_ROWS = 4;
 constexpr int MERGE_THREADS = 256;
-
-struct MergeW {
-  float wa, wb, inv, lse;
-  int mode;  // 0 normal, 1 both empty, 2 NaN
-};
-
-__device__ __forceinline__ MergeW merge_weights(float la, float lb) {
-  MergeW w;
-  if (isnan(la) || isnan(lb)) {
-    w.mode = 2;
-    w.wa = w.wb = w.inv = w.lse = __int_as_float(0x7fc00000);
-    return w;
-  }
-  const float mx = fmaxf(la, lb);
-  if (mx == -INFINITY) {
-    w.mode = 1;
-    w.wa = w.wb = 0.f;
-    w.inv = 0.f;
-    w.lse = -INFINITY;
-    return w;
-  }
-  w.mode = 0;
-  w.wa = expf(la - mx);
-  w.wb = expf(lb - mx);
-  const float den = __fadd_rn(w.wa, w.wb);
-  w.inv = __frcp_rn(den);
-  w.lse = mx + logf(den);
-  return w;
-}
-
-__device__ __forceinline__ float merge_one(const MergeW& w, float a, float b) {
-  if (w.mode == 1) return 0.f;
-  if (w.mode == 2) return w.lse;
-  const float ta = (w.wa == 0.f) ? 0.f : __fmul_rn(w.wa, a);
-  const float tb = (w.wb == 0.f) ? 0.f : __fmul_rn(w.wb, b);
-  return __fmul_rn(__fadd_rn(ta, tb), w.inv);
-}
 
 __global__ void __launch_bounds__(MERGE_THREADS) ra_merge_kernel(
     const float* o_a, const float* lse_a, const float* o_b, const float* lse_b, float* o_out,

@@ -46,7 +46,7 @@ def test_status_strings_and_version(lib):
                                  "RA_ERR_CUDA", "RA_ERR_TIMEOUT"]):
         assert _lib.status_string(code) == name
     assert _lib.status_string(99) == "RA_ERR_UNKNOWN"
-    assert _lib.ring_attn_version() == 100
+    assert _lib.ring_attn_version() == 101
 
 
 # Fake, never-dereferenced device addresses: validation rejects these calls
@@ -91,6 +91,45 @@ def test_fwd_rejects_invalid_arguments(lib, kw, status):
 @pytest.mark.parametrize("kw", [dict(B=0), dict(L=0), dict(Hq=0, Hkv=0)])
 def test_fwd_empty_problem_launches_nothing(lib, kw):
     assert fwd_status(lib, q=0, k=0, v=0, out=0, lse=0, **kw) == _lib.RA_OK
+
+
+OACC = 6 * A * 64
+
+
+def visit_status(lib, **kw):
+    args = dict(q=Q, k=K, v=V, o_acc=OACC, lse_acc=LSE, out=O, B=1, Hq=2, Hkv=2, l=512, d=128,
+                diag=1, fold=1, scale=0.088)
+    args.update(kw)
+    return lib.ring_attn_fwd_visit(args["q"], args["k"], args["v"], args["o_acc"],
+                                   args["lse_acc"], args["out"], args["B"], args["Hq"],
+                                   args["Hkv"], args["l"], args["d"], args["diag"], args["fold"],
+                                   args["scale"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(diag=3), _lib.RA_ERR_INVALID_ARG),
+    (dict(diag=-1), _lib.RA_ERR_INVALID_ARG),
+    (dict(fold=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.RA_ERR_INVALID_ARG),
+    (dict(d=96), _lib.RA_ERR_UNSUPPORTED),
+    (dict(o_acc=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(lse_acc=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(o_acc=OACC + 4), _lib.RA_ERR_INVALID_ARG),     # not 16-byte aligned
+    (dict(out=O + 8), _lib.RA_ERR_INVALID_ARG),
+    (dict(o_acc=Q + 64), _lib.RA_ERR_INVALID_ARG),      # accumulator overlaps q
+    (dict(out=OACC + 4096), _lib.RA_ERR_INVALID_ARG),   # out overlaps the accumulator
+    (dict(lse_acc=OACC + 16), _lib.RA_ERR_INVALID_ARG),
+    (dict(B=1, l=1 << 31), _lib.RA_ERR_INVALID_ARG),
+])
+def test_visit_rejects_invalid_arguments(lib, kw, status):
+    assert visit_status(lib, **kw) == status
+    assert _lib.last_error()
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(l=0), dict(Hq=0, Hkv=0)])
+def test_visit_empty_problem_launches_nothing(lib, kw):
+    assert visit_status(lib, q=0, k=0, v=0, o_acc=0, lse_acc=0, out=0, **kw) == _lib.RA_OK
 
 
 def merge_status(lib, rows=64, d=128, **kw):
