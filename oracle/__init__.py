@@ -16,6 +16,10 @@ are
 * "大模型底层原理注意力机制优化与长上下文处理" (lnwmold), §2.1 (standard
   self-attention) and §2.2 (MQA/GQA).
 
+``attn_fp64`` holds the forward pass and the ring; ``attn_bwd_fp64`` the
+gradients of the same definition (the backward pass the FlashAttention
+article's recomputation serves).
+
 Every function here has a pin in ``tests/test_oracle.py`` against something
 other than itself (a library routine, a closed form, an invariant, the pages'
 worked example, or brute force on tiny inputs); none is parity unpinned.
@@ -35,4 +39,9 @@ from .attn_fp64 import (  # noqa: F401
     merge,
     causal_pair_counts,
     kv_bytes_per_ring_step,
+)
+from .attn_bwd_fp64 import (  # noqa: F401
+    attention_bwd,
+    attention_bwd_dq_rows,
+    attention_bwd_kv_rows,
 )
