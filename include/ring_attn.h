@@ -19,12 +19,14 @@
  *     launched; device-side failures are reported by ring_attn_check_status.
  *   - No C++ exception crosses the ABI.  A non-OK status leaves a one-line
  *     explanation that ring_attn_last_error() returns (per host thread).
- *   - The library holds no device allocation of its own except one status
- *     word per device (a static device variable of the module).
+ *   - The library holds no device allocation of its own except two status
+ *     words per device (static device variables of the module: one for the
+ *     forward kernels, one for the backward kernels).
  */
 #ifndef RING_ATTN_H_
 #define RING_ATTN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -124,6 +126,50 @@ ra_status ring_attn_fwd_visit(const void* q, const void* k, const void* v, float
                               int diag, int fold, float scale, ra_stream_t stream);
 
 /*
+ * ring_attn_bwd_workspace_size -- bytes of device workspace ring_attn_bwd
+ * needs: one fp32 per query row and head (B * Hq * L * 4).
+ */
+ra_status ring_attn_bwd_workspace_size(int B, int Hq, int64_t L, size_t* bytes);
+
+/*
+ * ring_attn_bwd -- backward pass of ring_attn_fwd: the gradients of
+ * sum(out * dout) with respect to q, k and v, recomputing the attention
+ * weights from the forward's lse instead of storing them (FlashAttention
+ * article, section 二, 核心原理 / 重计算):
+ *     P  = exp(scale * Q K^T - lse)   (masked entries 0)
+ *     dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D)
+ *     dQ = scale * dS K,  dK = scale * dS^T Q
+ * with the K/V gradient of each grouped-query head summed over its group.
+ * The work follows the ring of "Ring Attention 环注意力" L4 §4.2: the query
+ * block of host i visits K/V blocks (i - t) mod n_ring and the K/V block of
+ * host j (with its dK, dV) visits query blocks (j + t) mod n_ring; causal
+ * visits of a later K/V block are skipped.  P and dS are rounded to bf16
+ * before their products (as P is in the forward), accumulation is fp32,
+ * outputs are rounded to nearest even.
+ *
+ *   q, k, v, scale, B, Hq, Hkv, L, d, n_ring, causal   exactly as given to
+ *          ring_attn_fwd (same layouts and limits)                    (in)
+ *   out    bf16 [B, L, Hq, d]: the forward output                     (in)
+ *   dout   bf16 [B, L, Hq, d]: the gradient of the loss w.r.t. out     (in)
+ *   lse    fp32 [B, Hq, L]: the forward lse                          (in)
+ *   dq     bf16 [B, L, Hq, d]                                        (out)
+ *   dk, dv bf16 [B, L, Hkv, d]                                       (out)
+ *   workspace  device memory of at least ring_attn_bwd_workspace_size
+ *          bytes, owned by the caller; holds D between the two kernels of
+ *          the call, so two calls in flight at once need two workspaces.
+ *
+ * Pointers must be 16-byte aligned; outputs and workspace must not overlap
+ * the inputs or each other.  B*Hq*L == 0 launches nothing.  Errors as for
+ * ring_attn_fwd, plus RA_ERR_INVALID_ARG for a short workspace.  Two kernels
+ * are launched on `stream` (dQ with D first, then dK/dV).
+ */
+ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                        int64_t L, int d, int n_ring, int causal, float scale,
+                        ra_stream_t stream);
+
+/*
  * ring_attn_merge -- fold two partial attention results over disjoint key
  * sets into one (the accumulation of each ring step's blockwise result into
  * O_i, "Ring Attention 环注意力" L4 §4.2 step 2, kept as output plus
@@ -148,8 +194,8 @@ ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b
 
 /*
  * ring_attn_check_status -- synchronise `stream`, then read and clear the
- * device status word of the current device.  Every device-side wait of the
- * forward kernel is bounded (see ring_attn_set_wait_limit_ns); a wait that
+ * device status words of the current device.  Every device-side wait of the
+ * forward and backward kernels is bounded (see ring_attn_set_wait_limit_ns); a wait that
  * runs out makes the kernel record RA_ERR_TIMEOUT, release its tensor memory
  * and return, leaving the CUDA context usable.  Returns RA_ERR_CUDA if the
  * synchronisation itself fails.
@@ -176,10 +222,10 @@ ra_status ring_attn_set_max_ctas(int n);
 enum { RA_SCHEDULE_AUTO = 0, RA_SCHEDULE_LONGEST_FIRST = 1, RA_SCHEDULE_HEAD_MAJOR = 2 };
 ra_status ring_attn_set_schedule(int schedule);
 
-/* Host-side fault injection for tests.  Bit 0: the forward kernel's loader
- * skips the first query-tile load, so the first bounded wait on it runs out
- * and the call reports RA_ERR_TIMEOUT through ring_attn_check_status.
- * 0 clears.  Process-wide. */
+/* Host-side fault injection for tests.  Bit 0: the loader of the forward
+ * kernel and of the backward dQ kernel skips its first query-tile load, so
+ * the first bounded wait on it runs out and the call reports RA_ERR_TIMEOUT
+ * through ring_attn_check_status.  0 clears.  Process-wide. */
 ra_status ring_attn_debug_inject(unsigned flags);
 
 /* Human-readable name of a status code (static storage). */

@@ -9,6 +9,8 @@ and the seeded synthetic inputs (``inputs``).
 
 from ._lib import (  # noqa: F401
     RingAttnError,
+    ring_attn_bwd,
+    ring_attn_bwd_workspace_size,
     ring_attn_check_status,
     ring_attn_debug_inject,
     ring_attn_fwd,

@@ -25,6 +25,9 @@ SIGNATURES = {
     "ring_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, ctypes.c_float, _P]),
     "ring_attn_fwd_visit": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I,
                                  ctypes.c_float, _P]),
+    "ring_attn_bwd_workspace_size": (_I, [_I, _I, _I64, ctypes.POINTER(ctypes.c_size_t)]),
+    "ring_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I64,
+                           _I, _I, _I, ctypes.c_float, _P]),
     "ring_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I, _P]),
     "ring_attn_check_status": (_I, [_P]),
     "ring_attn_set_wait_limit_ns": (_I, [ctypes.c_uint64]),
@@ -78,6 +81,19 @@ def _check(status: int) -> int:
 
 def ring_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, L, d, n_ring, causal, scale, stream=0):
     return _check(load().ring_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, L, d, n_ring,
+                                       int(bool(causal)), float(scale), stream))
+
+
+def ring_attn_bwd_workspace_size(B, Hq, L):
+    n = ctypes.c_size_t(0)
+    _check(load().ring_attn_bwd_workspace_size(B, Hq, L, ctypes.byref(n)))
+    return n.value
+
+
+def ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, L,
+                  d, n_ring, causal, scale, stream=0):
+    return _check(load().ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace,
+                                       workspace_bytes, B, Hq, Hkv, L, d, n_ring,
                                        int(bool(causal)), float(scale), stream))
 
 

@@ -52,6 +52,47 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: 
     return out, lse
 
 
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+        dout: torch.Tensor, lse: torch.Tensor, n_ring: int, causal: bool,
+        scale: float | None = None, dq: torch.Tensor | None = None,
+        dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+        workspace: torch.Tensor | None = None, stream=None):
+    """Backward pass of ``fwd``: q/k/v/n_ring/causal/scale as given to it, its
+    out (bf16 [B, L, Hq, d]) and lse (fp32 [B, Hq, L]), and dout (bf16, like
+    out).  Returns (dq, dk, dv) in bf16.  ``workspace`` (any CUDA tensor of at
+    least ``ring_attn_bwd_workspace_size`` bytes) is allocated if omitted."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check_cuda(t, n, torch.bfloat16, 4)
+    _check_cuda(lse, "lse", torch.float32, 3)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, L, Hkv, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
+    if out.shape != q.shape or dout.shape != q.shape or lse.shape != (B, Hq, L):
+        raise ValueError("out/dout/lse shapes do not match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _check_cuda(t, n, torch.bfloat16, 4)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} shape does not match")
+    need = _lib.ring_attn_bwd_workspace_size(B, Hq, L)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _lib.ring_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                           dv.data_ptr(), workspace.data_ptr(), ws_bytes, B, Hq, Hkv, L, d,
+                           n_ring, causal, scale, _stream_handle(stream))
+    return dq, dk, dv
+
+
 def fwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Tensor,
               lse_acc: torch.Tensor, diag: int, fold: bool, scale: float | None = None,
               out: torch.Tensor | None = None, stream=None):

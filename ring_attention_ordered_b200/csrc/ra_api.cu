@@ -239,6 +239,84 @@ ra_status ring_attn_fwd_visit(const void* q, const void* k, const void* v, float
                         diag != 0, scale, nkv, stream);
 }
 
+ra_status ring_attn_bwd_workspace_size(int B, int Hq, int64_t L, size_t* bytes) {
+  if (!bytes) return fail(RA_ERR_INVALID_ARG, "null size pointer");
+  if (B < 0 || Hq < 0 || L < 0) return fail(RA_ERR_INVALID_ARG, "negative size");
+  *bytes = static_cast<size_t>(B) * static_cast<size_t>(Hq) * static_cast<size_t>(L) * 4;
+  return ok();
+}
+
+ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                        int64_t L, int d, int n_ring, int causal, float scale,
+                        ra_stream_t stream) {
+  ra_status st = check_forward_shape(B, Hq, Hkv, L, d, n_ring, causal, scale);
+  if (st != RA_OK) return st;
+  if (static_cast<long long>(B) * Hq * L == 0) return ok();
+  const size_t nq = static_cast<size_t>(B) * L * Hq * d * 2;
+  const size_t nkv = static_cast<size_t>(B) * L * Hkv * d * 2;
+  const size_t nl = static_cast<size_t>(B) * Hq * L * 4;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !workspace)
+    return fail(RA_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[10] = {q, k, v, out, dout, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return fail(RA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (workspace_bytes < nl)
+    return fail(RA_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed",
+                workspace_bytes, nl);
+  const void* ins[6] = {q, k, v, out, dout, lse};
+  const size_t in_n[6] = {nq, nkv, nkv, nq, nq, nl};
+  const void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_n[4] = {nq, nkv, nkv, nl};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(outs[o], out_n[o], ins[i], in_n[i]))
+        return fail(RA_ERR_INVALID_ARG, "an output or the workspace overlaps an input");
+    for (int o2 = o + 1; o2 < 4; ++o2)
+      if (overlaps(outs[o], out_n[o], outs[o2], out_n[o2]))
+        return fail(RA_ERR_INVALID_ARG, "outputs and workspace overlap each other");
+  }
+  int sms = 0;
+  if ((st = device_info(&sms)) != RA_OK) return st;
+  ra::BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const long long rows = static_cast<long long>(B) * L;
+  if ((st = make_map(&prm.tm_q, q, Hq, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_k, k, Hkv, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_v, v, Hkv, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_do, dout, Hq, rows, d)) != RA_OK) return st;
+  prm.out = static_cast<const __nv_bfloat16*>(out);
+  prm.dout = static_cast<const __nv_bfloat16*>(dout);
+  prm.lse = lse;
+  prm.dvec = static_cast<float*>(workspace);
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.L = static_cast<int>(L);
+  prm.n_ring = n_ring;
+  prm.blk_len = static_cast<int>(L / n_ring);
+  prm.causal = causal;
+  prm.tiles_per_blk = (prm.blk_len + 127) / 128;
+  const long long uq = static_cast<long long>(B) * Hq * n_ring * prm.tiles_per_blk;
+  const long long ukv = static_cast<long long>(B) * Hkv * n_ring * prm.tiles_per_blk;
+  if (uq >= (1ll << 31)) return fail(RA_ERR_INVALID_ARG, "problem too large (%lld work units)", uq);
+  prm.units_dq = static_cast<int>(uq);
+  prm.units_kv = static_cast<int>(ukv);
+  prm.scale = scale;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.wait_limit_ns = g_wait_limit_ns.load();
+  prm.debug_flags = g_debug_flags.load();
+  cudaError_t e = ra::launch_bwd(prm, d, sms, g_max_ctas.load(),
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b,
                           const float* lse_b, float* o_out, float* lse_out, int64_t rows, int d,
                           ra_stream_t stream) {
@@ -271,9 +349,11 @@ ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b
 ra_status ring_attn_check_status(ra_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
-  unsigned long long v = 0;
+  unsigned long long v = 0, vb = 0;
   e = ra::read_and_clear_status(&v);
+  if (e == cudaSuccess) e = ra::read_and_clear_bwd_status(&vb);
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (v == 0) v = vb;
   if (v == 0) return ok();
   const unsigned code = static_cast<unsigned>(v >> 32);
   const unsigned site = static_cast<unsigned>((v >> 16) & 0xFFFF);
@@ -319,6 +399,6 @@ const char* ring_attn_status_string(ra_status s) {
 
 const char* ring_attn_last_error(void) { return g_last_error.c_str(); }
 
-int ring_attn_version(void) { return 101; }
+int ring_attn_version(void) { return 102; }
 
 }  // extern "C"

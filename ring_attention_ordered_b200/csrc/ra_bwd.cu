@@ -1,0 +1,968 @@
+// Backward pass of ring-ordered blockwise attention for sm_100a.
+//
+// What it computes: the gradients of the forward pass for an upstream
+// gradient dO, recomputing the attention weights from the stored logsumexp
+// instead of storing them (FlashAttention article, section 二: 核心原理 and
+// 重计算 -- only O and the softmax statistics are kept):
+//   P  = exp(scale * Q K^T - lse)          (per query row; masked entries 0)
+//   dV = P^T dO
+//   dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D)
+//   dQ = scale * dS K,  dK = scale * dS^T Q
+// (D equals rowsum(P * dP), the row term of the softmax Jacobian, because
+// O = P V.)  Grouped-query heads (lnwmold page §2.2) add their dK, dV into the
+// shared K/V head.  The work is ordered as the ring of "Ring Attention 环注意力"
+// (L4 §4.2): the query block of host i visits K/V blocks (i - t) mod N, and
+// the K/V block of host j visits query blocks (j + t) mod N -- the order in
+// which dK_j, dV_j would travel the ring; causal visits with a later K/V block
+// are skipped (L4 §4.5 limitation 2).
+//
+// How (B200 design): two persistent kernels, one CTA per SM, each with one
+// softmax warpgroup (warps 0-3, one TMEM lane = one tile row), a TMA loader
+// warp (4) and a tcgen05.mma warp (5).
+//   * ra_bwd_dq_kernel: a unit is one 128-row query tile of one head; it
+//     computes D for its rows (written to the workspace), then for every K/V
+//     tile S = Q K^T and dP = dO V^T into TMEM, P and dS in the softmax
+//     warps (dS as bf16 over dP), and dQ += dS K accumulated in TMEM.
+//   * ra_bwd_dkdv_kernel (after it, on the same stream): a unit is one
+//     128-key tile of one K/V head; for every query tile of every head of the
+//     group, S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T in the
+//     softmax warps (bf16, over S^T and dP^T), dV += P^T dO and dK += dS^T Q
+//     accumulated in TMEM: no atomics, every gradient is written once.
+//   P is rounded to bf16 once and that value feeds both dV and dS.
+//   Every mbarrier wait is bounded (ra_sync.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+#include "ra_internal.h"
+#include "ra_sync.cuh"
+#include "ring_attn.h"
+
+namespace ra {
+namespace bwd {
+
+constexpr int TM = 128;              // rows per tile (queries or keys)
+constexpr int BOX_COLS = 64;
+constexpr int BOX_BYTES = 128 * 128;
+constexpr int NUM_THREADS = 192;     // softmax warpgroup, loader warp, MMA warp
+constexpr int WARP_LOAD = 4;
+constexpr int WARP_MMA = 5;
+constexpr float LOG2E = 1.4426950408889634f;
+
+// Device status word of the backward kernels: 0 = ok, else (code << 32) | where.
+__device__ unsigned long long g_status = 0ull;
+
+enum Site : uint32_t {
+  SITE_KV_FULL = 17, SITE_KV_EMPTY, SITE_QD_FULL, SITE_QD_EMPTY, SITE_S_FULL, SITE_S_FREE,
+  SITE_DP_FULL, SITE_P_FULL, SITE_DS_FULL, SITE_ACC_DONE, SITE_ACC_FREE
+};
+
+__device__ __forceinline__ int unit_for_round(int k, int G, int c) {
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// S-like MMA over the head dimension (A, B both K-major): D/16 steps.
+template <int KK>
+struct KStep {
+  static constexpr uint32_t OFF = ((KK / 4) * BOX_BYTES + (KK % 4) * 32) >> 4;
+};
+template <int D>
+__device__ __forceinline__ void mma_kmajor(uint32_t d, uint32_t a, uint32_t b, uint32_t hi,
+                                           uint32_t idesc) {
+  if (elect_one()) mma_ss<KStep<0>::OFF, KStep<0>::OFF>(d, a, hi, b, hi, idesc, 0u);
+  if (elect_one()) mma_ss<KStep<1>::OFF, KStep<1>::OFF>(d, a, hi, b, hi, idesc, 1u);
+  if (elect_one()) mma_ss<KStep<2>::OFF, KStep<2>::OFF>(d, a, hi, b, hi, idesc, 1u);
+  if (elect_one()) mma_ss<KStep<3>::OFF, KStep<3>::OFF>(d, a, hi, b, hi, idesc, 1u);
+  if constexpr (D == 128) {
+    if (elect_one()) mma_ss<KStep<4>::OFF, KStep<4>::OFF>(d, a, hi, b, hi, idesc, 1u);
+    if (elect_one()) mma_ss<KStep<5>::OFF, KStep<5>::OFF>(d, a, hi, b, hi, idesc, 1u);
+    if (elect_one()) mma_ss<KStep<6>::OFF, KStep<6>::OFF>(d, a, hi, b, hi, idesc, 1u);
+    if (elect_one()) mma_ss<KStep<7>::OFF, KStep<7>::OFF>(d, a, hi, b, hi, idesc, 1u);
+  }
+}
+
+// Accumulating MMA with A (bf16 pairs, 128 along K) in TMEM and B MN-major in
+// shared memory (K = 128 rows of 128 bytes per 64-column box): 8 steps of
+// 16, A advancing 8 columns, B 16 rows (2048 bytes) per step.
+__device__ __forceinline__ void mma_tmem_a(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t hi,
+                                           uint32_t idesc, uint32_t acc) {
+  if (elect_one()) mma_ts<0, 0>(d, a_tmem, b, hi, idesc, acc);
+  if (elect_one()) mma_ts<8, 128>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<16, 256>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<24, 384>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<32, 512>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<40, 640>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<48, 768>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<56, 896>(d, a_tmem, b, hi, idesc, 1u);
+}
+
+__device__ __forceinline__ void commit(uint32_t bar) {
+  if (elect_one()) tc_commit(bar);
+}
+
+// Store one row of fp32 accumulator columns [col0, col0 + D) of TMEM, times
+// `mul`, as bf16 to dst (D contiguous elements); all lanes load, only
+// `valid` lanes store.
+template <int D>
+__device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst,
+                                              bool valid) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32(taddr + cc * 32, o);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * mul, __uint_as_float(o[2 * j + 1]) * mul);
+    if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
+  }
+}
+
+// dS over 32 columns: ds = p * (dp - D), p from bf16 pairs pk (16 words), dp
+// from TMEM (fp32), D per column (dkdv: one per query, from shared memory)
+// or one for the whole row (dq: the row's own D).
+template <bool PER_COLUMN>
+__device__ __forceinline__ void ds_chunk(const uint32_t (&pk)[16], const uint32_t (&dp)[32],
+                                         const float* dcol, float drow, uint32_t (&out)[16]) {
+  const uint64_t dr2 = f2_pack(drow, drow);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint64_t p2 = f2_pack(bf16lo(pk[j]), bf16hi(pk[j]));
+    const uint64_t dd = PER_COLUMN ? f2_pack(dcol[2 * j], dcol[2 * j + 1]) : dr2;
+    const uint64_t d2 =
+        f2_sub(f2_pack(__uint_as_float(dp[2 * j]), __uint_as_float(dp[2 * j + 1])), dd);
+    float a, b;
+    f2_unpack(f2_mul(p2, d2), a, b);
+    out[j] = pack_bf16x2(a, b);
+  }
+}
+
+// =====================================================================
+// dQ kernel: query-stationary
+// =====================================================================
+template <int D>
+struct QCfg {
+  static constexpr int TILE = TM * D * 2;
+  static constexpr int NS = (D == 128) ? 2 : 4;       // K/V stages (K and V tile each)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE;
+  static constexpr int OFF_KV = 2 * TILE;
+  static constexpr int OFF_BAR = OFF_KV + NS * 2 * TILE;
+  // qo_full, qo_empty, kv_full[NS], kv_empty[NS], s_full, s_free, dp_full,
+  // ds_full, acc_done, acc_free, drain
+  static constexpr int NUM_BARS = 2 + 2 * NS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct QBars {
+  uint32_t base;
+  int ns;
+  __device__ __forceinline__ uint32_t qo_full() const { return base; }
+  __device__ __forceinline__ uint32_t qo_empty() const { return base + 8; }
+  __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 16 + 8u * s; }
+  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 16 + 8u * (ns + s); }
+  __device__ __forceinline__ uint32_t s_full() const { return base + 16 + 16u * ns; }
+  __device__ __forceinline__ uint32_t s_free() const { return s_full() + 8; }
+  __device__ __forceinline__ uint32_t dp_full() const { return s_full() + 16; }
+  __device__ __forceinline__ uint32_t ds_full() const { return s_full() + 24; }
+  __device__ __forceinline__ uint32_t acc_done() const { return s_full() + 32; }
+  __device__ __forceinline__ uint32_t acc_free() const { return s_full() + 40; }
+  __device__ __forceinline__ uint32_t drain() const { return s_full() + 48; }
+};
+
+struct QUnit {
+  int b, h, blk, qt, n;
+};
+
+// Units in (batch, head) order, longest first inside a head: the query block
+// i from last to first, its tiles from last to first.
+__device__ __forceinline__ QUnit q_unit(const BwdParams& p, int u) {
+  const int per_head = p.n_ring * p.tiles_per_blk;
+  const int bh = u / per_head;
+  const int rem = u - bh * per_head;
+  QUnit x;
+  x.b = bh / p.Hq;
+  x.h = bh - x.b * p.Hq;
+  x.blk = p.n_ring - 1 - rem / p.tiles_per_blk;
+  x.qt = p.tiles_per_blk - 1 - rem % p.tiles_per_blk;
+  x.n = p.causal ? (x.blk * p.tiles_per_blk + x.qt + 1) : p.n_ring * p.tiles_per_blk;
+  return x;
+}
+
+// K/V tiles of a query unit in ring order: own block first (tiles 0..qt
+// under causal masking), then blocks blk-1, blk-2, ... wrapping around.
+struct KvWalk {
+  int jb, kl, end;
+  __device__ __forceinline__ void start(const BwdParams& p, const QUnit& x) {
+    jb = x.blk;
+    kl = 0;
+    end = p.causal ? x.qt + 1 : p.tiles_per_blk;
+  }
+  __device__ __forceinline__ void next(const BwdParams& p) {
+    if (++kl == end) {
+      kl = 0;
+      jb = (jb == 0) ? p.n_ring - 1 : jb - 1;
+      end = p.tiles_per_blk;
+    }
+  }
+};
+
+template <int D>
+__device__ void dq_loader(const BwdParams& p, const QBars& br, uint32_t base, const Ctl& cx) {
+  using C = QCfg<D>;
+  constexpr int NBOX = D / BOX_COLS;
+  const int G = gridDim.x, c = blockIdx.x;
+  uint32_t kv_it = 0, units = 0;
+  bool qo_pending = false;
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
+    if (u >= p.units_dq) break;
+    const QUnit x = q_unit(p, u);
+    if (units > 0 && !wait_warp(br.qo_empty(), (units - 1) & 1u, cx, SITE_QD_EMPTY)) goto drain;
+    if ((p.debug_flags & 1u) && units == 0) {
+      // fault injection: the first query tiles are never requested
+    } else {
+      const int row = x.b * p.L + x.blk * p.blk_len + x.qt * TM;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.qo_full(), 2 * C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+          tma_load_3d(base + C::OFF_Q + bx * BOX_BYTES, &p.tm_q, br.qo_full(), bx * BOX_COLS, x.h, row);
+          tma_load_3d(base + C::OFF_DO + bx * BOX_BYTES, &p.tm_do, br.qo_full(), bx * BOX_COLS, x.h,
+                      row);
+        }
+      }
+      __syncwarp();
+      qo_pending = true;
+    }
+    ++units;
+    KvWalk it;
+    it.start(p, x);
+    const int kvh = x.h / p.group;
+    for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
+      const int s = kv_it % C::NS;
+      const uint32_t ph = (kv_it / C::NS) & 1u;
+      if (!wait_warp(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
+      const int row = x.b * p.L + it.jb * p.blk_len + it.kl * TM;
+      const uint32_t dst = base + C::OFF_KV + s * 2 * C::TILE;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.kv_full(s), 2 * C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+          tma_load_3d(dst + bx * BOX_BYTES, &p.tm_k, br.kv_full(s), bx * BOX_COLS, kvh, row);
+          tma_load_3d(dst + C::TILE + bx * BOX_BYTES, &p.tm_v, br.kv_full(s), bx * BOX_COLS, kvh,
+                      row);
+        }
+      }
+      __syncwarp();
+      ++kv_it;
+    }
+  }
+  return;
+drain:
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t n = kv_it < static_cast<uint32_t>(C::NS) ? kv_it : C::NS;
+    for (uint32_t i = 0; i < n; ++i) {
+      const uint32_t it = kv_it - 1 - i;
+      drain_wait(br.kv_full(it % C::NS), (it / C::NS) & 1u, 200000000ull);
+    }
+    if (qo_pending) drain_wait(br.qo_full(), (units - 1) & 1u, 200000000ull);
+  }
+  __syncwarp();
+}
+
+template <int D>
+__device__ void dq_mma(const BwdParams& p, const QBars& br, uint32_t base, uint32_t tmem,
+                       const Ctl& cx) {
+  using C = QCfg<D>;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(TM, TM, false);
+  constexpr uint32_t IDESC_DQ = idesc_bf16_f32(TM, D, true);
+  const int G = gridDim.x, c = blockIdx.x;
+  const uint64_t dq0 = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
+  const uint64_t ddo0 = smem_desc_sw128(base + C::OFF_DO, 16, 1024);
+  const uint64_t dk0 = smem_desc_sw128(base + C::OFF_KV, 16, 1024);
+  const uint64_t dkmn0 = smem_desc_sw128(base + C::OFF_KV, BOX_BYTES, 1024);
+  const uint32_t q_lo = static_cast<uint32_t>(dq0), do_lo = static_cast<uint32_t>(ddo0);
+  const uint32_t k_lo = static_cast<uint32_t>(dk0), kmn_lo = static_cast<uint32_t>(dkmn0);
+  const uint32_t hi = static_cast<uint32_t>(dk0 >> 32), mn_hi = static_cast<uint32_t>(dkmn0 >> 32);
+  const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+  uint32_t kv_it = 0, units = 0, step = 0;
+  auto issue_s = [&](int s) {
+    mma_kmajor<D>(t_s, q_lo, k_lo + ((s * 2 * C::TILE) >> 4), hi, IDESC_S);
+  };
+  auto issue_dp = [&](int s) {
+    mma_kmajor<D>(t_dp, do_lo, k_lo + ((s * 2 * C::TILE + C::TILE) >> 4), hi, IDESC_S);
+  };
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
+    if (u >= p.units_dq) break;
+    const QUnit x = q_unit(p, u);
+    const int n = x.n;
+    if (!wait_warp(br.qo_full(), units & 1u, cx, SITE_QD_FULL)) goto drain;
+    {
+      const int s = kv_it % C::NS;
+      if (!wait_warp(br.kv_full(s), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+      tc_fence_after();
+      issue_s(s);
+      commit(br.s_full());
+      issue_dp(s);
+      commit(br.dp_full());
+    }
+    for (int idx = 0; idx < n; ++idx) {
+      const bool more = idx + 1 < n;
+      const int s = kv_it % C::NS;
+      const int s1 = (kv_it + 1) % C::NS;
+      if (more) {
+        // S for the next K/V tile as soon as the softmax has read this one
+        if (!wait_warp(br.s_free(), step & 1u, cx, SITE_S_FREE)) goto drain;
+        if (!wait_warp(br.kv_full(s1), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+        tc_fence_after();
+        issue_s(s1);
+        commit(br.s_full());
+      }
+      if (!wait_warp(br.ds_full(), step & 1u, cx, SITE_DS_FULL)) goto drain;
+      if (idx == 0 && units > 0 &&
+          !wait_warp(br.acc_free(), (units - 1) & 1u, cx, SITE_ACC_FREE))
+        goto drain;
+      tc_fence_after();
+      mma_tmem_a(t_dq, t_dp, kmn_lo + ((s * 2 * C::TILE) >> 4), mn_hi, IDESC_DQ, idx > 0 ? 1u : 0u);
+      commit(br.kv_empty(s));
+      if (more) {
+        issue_dp(s1);
+        commit(br.dp_full());
+      }
+      ++step;
+      ++kv_it;
+    }
+    commit(br.acc_done());
+    commit(br.qo_empty());
+    ++units;
+  }
+  return;
+drain:
+  commit(br.drain());
+  if ((threadIdx.x & 31) == 0) drain_wait(br.drain(), 0u, 200000000ull);
+  __syncwarp();
+}
+
+template <int D>
+__device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, const Ctl& cx) {
+  const int t = threadIdx.x;                       // row inside the query tile
+  const int quarter = t >> 5;
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t t_s = tmem + lane_off, t_dp = t_s + 128, t_dq = t_s + 256;
+  const float c2 = p.scale_log2;
+  const int G = gridDim.x, c = blockIdx.x;
+  uint32_t units = 0, step = 0;
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
+    if (u >= p.units_dq) break;
+    const QUnit x = q_unit(p, u);
+    const int qrow = x.qt * TM + t;
+    const bool valid = qrow < p.blk_len;
+    const long long grow = static_cast<long long>(x.blk) * p.blk_len + qrow;
+    const long long vidx = (static_cast<long long>(x.b) * p.Hq + x.h) * p.L + grow;
+    // D = rowsum(dO * O) of this row, and the row's lse in base 2
+    float dvec = 0.f, nlse2 = -INFINITY;
+    if (valid) {
+      const long long off = ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D;
+      const uint4* o4 = reinterpret_cast<const uint4*>(p.out + off);
+      const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + off);
+      float acc = 0.f;
+#pragma unroll 4
+      for (int j = 0; j < D / 8; ++j) {
+        const uint4 a = o4[j], g = g4[j];
+        acc = fmaf(bf16lo(a.x), bf16lo(g.x), acc);
+        acc = fmaf(bf16hi(a.x), bf16hi(g.x), acc);
+        acc = fmaf(bf16lo(a.y), bf16lo(g.y), acc);
+        acc = fmaf(bf16hi(a.y), bf16hi(g.y), acc);
+        acc = fmaf(bf16lo(a.z), bf16lo(g.z), acc);
+        acc = fmaf(bf16hi(a.z), bf16hi(g.z), acc);
+        acc = fmaf(bf16lo(a.w), bf16lo(g.w), acc);
+        acc = fmaf(bf16hi(a.w), bf16hi(g.w), acc);
+      }
+      dvec = acc;
+      p.dvec[vidx] = acc;
+      nlse2 = -p.lse[vidx] * LOG2E;
+    }
+    const uint64_t nl2 = f2_pack(nlse2, nlse2);
+    const uint64_t c2x2 = f2_pack(c2, c2);
+
+    KvWalk it;
+    it.start(p, x);
+    for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
+      int lim = min(TM, p.blk_len - it.kl * TM) - 1;
+      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * TM);
+      const bool masked = __any_sync(0xffffffffu, lim < TM - 1);
+      if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(br.s_free());
+      // P = 2^(s * scale * log2 e - lse * log2 e), rounded to bf16 pairs
+      uint32_t pk[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        float e0, e1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), c2x2,
+                         nl2),
+                  e0, e1);
+        float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+        if (masked) {
+          p0 = (2 * j > lim) ? 0.f : p0;
+          p1 = (2 * j + 1 > lim) ? 0.f : p1;
+        }
+        pk[j] = pack_bf16x2(p0, p1);
+      }
+      if (!wait_warp(br.dp_full(), step & 1u, cx, SITE_DP_FULL)) return;
+      tc_fence_after();
+      // dS = P (dP - D) in four chunks of 32 keys, each stored as 16 columns
+      // of bf16 pairs over dP columns that have already been read
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dp[32];
+        tmem_ld32(t_dp + 32 * cc, dp);
+        tmem_wait_ld();
+        uint32_t ds[16];
+        ds_chunk<false>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp, nullptr, dvec,
+                        ds);
+        tmem_st16(t_dp + 16 * cc, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(br.ds_full());
+      ++step;
+    }
+    // epilogue: dQ = scale * (dS K) accumulated in TMEM
+    if (!wait_warp(br.acc_done(), units & 1u, cx, SITE_ACC_DONE)) return;
+    tc_fence_after();
+    __nv_bfloat16* dst = p.dq + ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D;
+    store_acc_row<D>(t_dq, p.scale, dst, valid);
+    tc_fence_before();
+    mbar_arrive(br.acc_free());
+    ++units;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  using C = QCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gen = smem_raw + (base - raw);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gen + C::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gen + C::OFF_MISC + 4);
+  const QBars br{base + C::OFF_BAR, C::NS};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    mbar_init(br.qo_full(), 1);
+    mbar_init(br.qo_empty(), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(br.kv_full(s), 1);
+      mbar_init(br.kv_empty(s), 1);
+    }
+    mbar_init(br.s_full(), 1);
+    mbar_init(br.s_free(), 128);
+    mbar_init(br.dp_full(), 1);
+    mbar_init(br.ds_full(), 128);
+    mbar_init(br.acc_done(), 1);
+    mbar_init(br.acc_free(), 128);
+    mbar_init(br.drain(), 1);
+    *abort_flag = 0u;
+    fence_mbarrier_init();
+  }
+  if (warp == WARP_LOAD && lane == 0) {
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_do);
+    prefetch_tensormap(&p.tm_k);
+    prefetch_tensormap(&p.tm_v);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
+  if (warp < 4) {
+    dq_softmax<D>(p, br, tmem, cx);
+  } else if (warp == WARP_LOAD) {
+    dq_loader<D>(p, br, base, cx);
+  } else {
+    dq_mma<D>(p, br, base, tmem, cx);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =====================================================================
+// dK/dV kernel: key-stationary
+// =====================================================================
+template <int D>
+struct KCfg {
+  static constexpr int TILE = TM * D * 2;
+  static constexpr int NS = (D == 128) ? 2 : 4;       // Q/dO stages
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_ST = 2 * TILE;             // stage s: Q, then dO
+  static constexpr int OFF_VEC = OFF_ST + NS * 2 * TILE;  // stage s: -lse*log2e [128], D [128]
+  static constexpr int VEC_BYTES = 2 * TM * 4;
+  static constexpr int OFF_BAR = OFF_VEC + NS * VEC_BYTES;
+  // kv_full, kv_empty, qd_full[NS], qd_empty[NS], s_full, dp_full, p_full,
+  // ds_full, acc_done, acc_free, drain
+  static constexpr int NUM_BARS = 2 + 2 * NS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct KBars {
+  uint32_t base;
+  int ns;
+  __device__ __forceinline__ uint32_t kv_full() const { return base; }
+  __device__ __forceinline__ uint32_t kv_empty() const { return base + 8; }
+  __device__ __forceinline__ uint32_t qd_full(int s) const { return base + 16 + 8u * s; }
+  __device__ __forceinline__ uint32_t qd_empty(int s) const { return base + 16 + 8u * (ns + s); }
+  __device__ __forceinline__ uint32_t s_full() const { return base + 16 + 16u * ns; }
+  __device__ __forceinline__ uint32_t dp_full() const { return s_full() + 8; }
+  __device__ __forceinline__ uint32_t p_full() const { return s_full() + 16; }
+  __device__ __forceinline__ uint32_t ds_full() const { return s_full() + 24; }
+  __device__ __forceinline__ uint32_t acc_done() const { return s_full() + 32; }
+  __device__ __forceinline__ uint32_t acc_free() const { return s_full() + 40; }
+  __device__ __forceinline__ uint32_t drain() const { return s_full() + 48; }
+};
+
+struct KUnit {
+  int b, kvh, jb, kt, n;
+};
+
+// Units in (batch, K/V head) order, longest first inside a head: K/V block
+// j from first to last (a causal K/V block is seen by blocks j..N-1), its
+// tiles from first to last.
+__device__ __forceinline__ KUnit kv_unit(const BwdParams& p, int u) {
+  const int tpb = p.tiles_per_blk;
+  const int per_head = p.n_ring * tpb;
+  const int bh = u / per_head;
+  const int rem = u - bh * per_head;
+  KUnit x;
+  x.b = bh / p.Hkv;
+  x.kvh = bh - x.b * p.Hkv;
+  x.jb = rem / tpb;
+  x.kt = rem - x.jb * tpb;
+  x.n = p.group * (p.causal ? ((tpb - x.kt) + (p.n_ring - 1 - x.jb) * tpb) : p.n_ring * tpb);
+  return x;
+}
+
+// Query tiles of a K/V unit: blocks i = jb, jb+1, ... (wrapping when not
+// causal), within each the heads of the group, within each the tiles (in the
+// own block under causal masking only tiles kt.. see this key tile).
+struct QWalk {
+  int t, i, hh, qt, qt0;
+  __device__ __forceinline__ void start(const BwdParams& p, const KUnit& x) {
+    t = 0;
+    i = x.jb;
+    hh = 0;
+    qt0 = p.causal ? x.kt : 0;
+    qt = qt0;
+  }
+  __device__ __forceinline__ void next(const BwdParams& p) {
+    if (++qt < p.tiles_per_blk) return;
+    if (++hh < p.group) {
+      qt = qt0;
+      return;
+    }
+    hh = 0;
+    ++t;
+    i = (i + 1 == p.n_ring) ? 0 : i + 1;
+    qt0 = 0;
+    qt = 0;
+  }
+};
+
+template <int D>
+__device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, float* vec_smem,
+                          const Ctl& cx) {
+  using C = KCfg<D>;
+  constexpr int NBOX = D / BOX_COLS;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  uint32_t q_it = 0, units = 0;
+  bool kv_pending = false;
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
+    if (u >= p.units_kv) break;
+    const KUnit x = kv_unit(p, u);
+    if (units > 0 && !wait_warp(br.kv_empty(), (units - 1) & 1u, cx, SITE_KV_EMPTY)) goto drain;
+    {
+      const int row = x.b * p.L + x.jb * p.blk_len + x.kt * TM;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.kv_full(), 2 * C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+          tma_load_3d(base + C::OFF_K + bx * BOX_BYTES, &p.tm_k, br.kv_full(), bx * BOX_COLS, x.kvh, row);
+          tma_load_3d(base + C::OFF_V + bx * BOX_BYTES, &p.tm_v, br.kv_full(), bx * BOX_COLS, x.kvh, row);
+        }
+      }
+      __syncwarp();
+      kv_pending = true;
+    }
+    ++units;
+    QWalk it;
+    it.start(p, x);
+    for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
+      const int s = q_it % C::NS;
+      const uint32_t ph = (q_it / C::NS) & 1u;
+      if (!wait_warp(br.qd_empty(s), ph ^ 1u, cx, SITE_QD_EMPTY)) goto drain;
+      const int h = x.kvh * p.group + it.hh;
+      const int row = x.b * p.L + it.i * p.blk_len + it.qt * TM;
+      const uint32_t dst = base + C::OFF_ST + s * 2 * C::TILE;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.qd_full(s), 2 * C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx) {
+          tma_load_3d(dst + bx * BOX_BYTES, &p.tm_q, br.qd_full(s), bx * BOX_COLS, h, row);
+          tma_load_3d(dst + C::TILE + bx * BOX_BYTES, &p.tm_do, br.qd_full(s), bx * BOX_COLS, h, row);
+        }
+      }
+      // -lse * log2(e) and D of the tile's 128 query rows (rows past the
+      // block end: weight 0 through -inf, D = 0)
+      float* vs = vec_smem + s * 2 * TM;
+      const long long vbase = (static_cast<long long>(x.b) * p.Hq + h) * p.L +
+                              static_cast<long long>(it.i) * p.blk_len;
+#pragma unroll
+      for (int j = 0; j < TM / 32; ++j) {
+        const int r = lane + 32 * j;
+        const int qrow = it.qt * TM + r;
+        float nl = -INFINITY, dvv = 0.f;
+        if (qrow < p.blk_len) {
+          nl = -p.lse[vbase + qrow] * LOG2E;
+          dvv = p.dvec[vbase + qrow];
+        }
+        vs[r] = nl;
+        vs[TM + r] = dvv;
+      }
+      mbar_arrive(br.qd_full(s));
+      ++q_it;
+    }
+  }
+  return;
+drain:
+  if (lane == 0) {
+    const uint32_t n = q_it < static_cast<uint32_t>(C::NS) ? q_it : C::NS;
+    for (uint32_t i = 0; i < n; ++i) {
+      const uint32_t it = q_it - 1 - i;
+      drain_wait(br.qd_full(it % C::NS), (it / C::NS) & 1u, 200000000ull);
+    }
+    if (kv_pending) drain_wait(br.kv_full(), (units - 1) & 1u, 200000000ull);
+  }
+  __syncwarp();
+}
+
+template <int D>
+__device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint32_t tmem,
+                       const Ctl& cx) {
+  using C = KCfg<D>;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(TM, TM, false);
+  constexpr uint32_t IDESC_ACC = idesc_bf16_f32(TM, D, true);
+  const int G = gridDim.x, c = blockIdx.x;
+  const uint64_t dk0 = smem_desc_sw128(base + C::OFF_K, 16, 1024);
+  const uint64_t dv0 = smem_desc_sw128(base + C::OFF_V, 16, 1024);
+  const uint64_t dst0 = smem_desc_sw128(base + C::OFF_ST, 16, 1024);
+  const uint64_t dstmn0 = smem_desc_sw128(base + C::OFF_ST, BOX_BYTES, 1024);
+  const uint32_t k_lo = static_cast<uint32_t>(dk0), v_lo = static_cast<uint32_t>(dv0);
+  const uint32_t st_lo = static_cast<uint32_t>(dst0), stmn_lo = static_cast<uint32_t>(dstmn0);
+  const uint32_t hi = static_cast<uint32_t>(dk0 >> 32), mn_hi = static_cast<uint32_t>(dstmn0 >> 32);
+  const uint32_t t_s = tmem, t_dp = tmem + 128, t_dv = tmem + 256, t_dk = tmem + 256 + D;
+  uint32_t q_it = 0, units = 0, step = 0;
+  // S^T = K Q^T and dP^T = V dO^T for stage s (Q and dO K-major)
+  auto issue_s = [&](int s) {
+    mma_kmajor<D>(t_s, k_lo, st_lo + ((s * 2 * C::TILE) >> 4), hi, IDESC_S);
+  };
+  auto issue_dp = [&](int s) {
+    mma_kmajor<D>(t_dp, v_lo, st_lo + ((s * 2 * C::TILE + C::TILE) >> 4), hi, IDESC_S);
+  };
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
+    if (u >= p.units_kv) break;
+    const KUnit x = kv_unit(p, u);
+    const int n = x.n;
+    if (!wait_warp(br.kv_full(), units & 1u, cx, SITE_KV_FULL)) goto drain;
+    {
+      const int s = q_it % C::NS;
+      if (!wait_warp(br.qd_full(s), (q_it / C::NS) & 1u, cx, SITE_QD_FULL)) goto drain;
+      tc_fence_after();
+      issue_s(s);
+      commit(br.s_full());
+      issue_dp(s);
+      commit(br.dp_full());
+    }
+    for (int idx = 0; idx < n; ++idx) {
+      const bool more = idx + 1 < n;
+      const int s = q_it % C::NS;
+      const int s1 = (q_it + 1) % C::NS;
+      if (!wait_warp(br.p_full(), step & 1u, cx, SITE_P_FULL)) goto drain;
+      if (idx == 0 && units > 0 &&
+          !wait_warp(br.acc_free(), (units - 1) & 1u, cx, SITE_ACC_FREE))
+        goto drain;
+      tc_fence_after();
+      // dV += P^T dO (dO MN-major)
+      mma_tmem_a(t_dv, t_s, stmn_lo + ((s * 2 * C::TILE + C::TILE) >> 4), mn_hi, IDESC_ACC,
+                 idx > 0 ? 1u : 0u);
+      if (more) {
+        // S^T of the next step may overwrite P^T: the tensor pipe runs the
+        // MMAs in order, so dV has read it by then
+        if (!wait_warp(br.qd_full(s1), ((q_it + 1) / C::NS) & 1u, cx, SITE_QD_FULL)) goto drain;
+        tc_fence_after();
+        issue_s(s1);
+        commit(br.s_full());
+      }
+      if (!wait_warp(br.ds_full(), step & 1u, cx, SITE_DS_FULL)) goto drain;
+      tc_fence_after();
+      // dK += dS^T Q (Q MN-major)
+      mma_tmem_a(t_dk, t_dp, stmn_lo + ((s * 2 * C::TILE) >> 4), mn_hi, IDESC_ACC,
+                 idx > 0 ? 1u : 0u);
+      commit(br.qd_empty(s));
+      if (more) {
+        issue_dp(s1);
+        commit(br.dp_full());
+      }
+      ++step;
+      ++q_it;
+    }
+    commit(br.acc_done());
+    commit(br.kv_empty());
+    ++units;
+  }
+  return;
+drain:
+  commit(br.drain());
+  if ((threadIdx.x & 31) == 0) drain_wait(br.drain(), 0u, 200000000ull);
+  __syncwarp();
+}
+
+template <int D>
+__device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, const float* vec_smem,
+                           const Ctl& cx) {
+  using C = KCfg<D>;
+  const int t = threadIdx.x;                       // key row inside the tile
+  const int quarter = t >> 5;
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t t_s = tmem + lane_off, t_dp = t_s + 128;
+  const uint32_t t_dv = t_s + 256, t_dk = t_s + 256 + D;
+  const uint64_t c2x2 = f2_pack(p.scale_log2, p.scale_log2);
+  const int G = gridDim.x, c = blockIdx.x;
+  uint32_t units = 0, step = 0, q_it = 0;
+  for (int k = 0;; ++k) {
+    const int u = unit_for_round(k, G, c);
+    if (u >= p.units_kv) break;
+    const KUnit x = kv_unit(p, u);
+    QWalk it;
+    it.start(p, x);
+    for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
+      const int s = q_it % C::NS;
+      // the diagonal tile of the own block: query column j sees key row t
+      // only when j >= t
+      const bool diag = p.causal && it.i == x.jb && it.qt == x.kt;
+      if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
+      // the loader's -lse and D for this stage are visible once its phase
+      // completed (it completed before S^T was issued)
+      if (!wait_warp(br.qd_full(s), (q_it / C::NS) & 1u, cx, SITE_QD_FULL)) return;
+      tc_fence_after();
+      const float* nl = vec_smem + s * 2 * TM;
+      const float* dvv = nl + TM;
+      uint32_t sr[128];
+      tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      uint32_t pk[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const float2 l2 = reinterpret_cast<const float2*>(nl)[j];
+        float e0, e1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), c2x2,
+                         f2_pack(l2.x, l2.y)),
+                  e0, e1);
+        float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+        if (diag) {
+          p0 = (2 * j < t) ? 0.f : p0;
+          p1 = (2 * j + 1 < t) ? 0.f : p1;
+        }
+        pk[j] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(t_s, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(t_s + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(br.p_full());
+      if (!wait_warp(br.dp_full(), step & 1u, cx, SITE_DP_FULL)) return;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dp[32];
+        tmem_ld32(t_dp + 32 * cc, dp);
+        tmem_wait_ld();
+        uint32_t ds[16];
+        ds_chunk<true>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp, dvv + 32 * cc,
+                       0.f, ds);
+        tmem_st16(t_dp + 16 * cc, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(br.ds_full());
+      ++step;
+      ++q_it;
+    }
+    // epilogue: dV and dK = scale * (dS^T Q) of this key tile
+    if (!wait_warp(br.acc_done(), units & 1u, cx, SITE_ACC_DONE)) return;
+    tc_fence_after();
+    const int krow = x.kt * TM + t;
+    const bool valid = krow < p.blk_len;
+    const long long off =
+        ((static_cast<long long>(x.b) * p.L + static_cast<long long>(x.jb) * p.blk_len + krow) * p.Hkv +
+         x.kvh) * D;
+    store_acc_row<D>(t_dv, 1.f, p.dv + off, valid);
+    store_acc_row<D>(t_dk, p.scale, p.dk + off, valid);
+    tc_fence_before();
+    mbar_arrive(br.acc_free());
+    ++units;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+  using C = KCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gen = smem_raw + (base - raw);
+  float* vec_smem = reinterpret_cast<float*>(gen + C::OFF_VEC);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gen + C::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gen + C::OFF_MISC + 4);
+  const KBars br{base + C::OFF_BAR, C::NS};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    mbar_init(br.kv_full(), 1);
+    mbar_init(br.kv_empty(), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(br.qd_full(s), 1 + 32);   // TMA transaction arrive + 32 loader lanes
+      mbar_init(br.qd_empty(s), 1);
+    }
+    mbar_init(br.s_full(), 1);
+    mbar_init(br.dp_full(), 1);
+    mbar_init(br.p_full(), 128);
+    mbar_init(br.ds_full(), 128);
+    mbar_init(br.acc_done(), 1);
+    mbar_init(br.acc_free(), 128);
+    mbar_init(br.drain(), 1);
+    *abort_flag = 0u;
+    fence_mbarrier_init();
+  }
+  if (warp == WARP_LOAD && lane == 0) {
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_do);
+    prefetch_tensormap(&p.tm_k);
+    prefetch_tensormap(&p.tm_v);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
+  if (warp < 4) {
+    kv_softmax<D>(p, br, tmem, vec_smem, cx);
+  } else if (warp == WARP_LOAD) {
+    kv_loader<D>(p, br, base, vec_smem, cx);
+  } else {
+    kv_mma<D>(p, br, base, tmem, cx);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+static cudaError_t launch_bwd_d(const BwdParams& prm, int num_sms, int max_ctas,
+                                cudaStream_t stream) {
+  static int configured_dev[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured_dev[dev]) {
+    e = cudaFuncSetAttribute(ra_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             QCfg<D>::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(ra_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             KCfg<D>::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured_dev[dev] = 1;
+  }
+  auto grid_for = [&](int units) {
+    int g = num_sms;
+    if (max_ctas > 0 && max_ctas < g) g = max_ctas;
+    return units < g ? units : g;
+  };
+  ra_bwd_dq_kernel<D><<<grid_for(prm.units_dq), NUM_THREADS, QCfg<D>::SMEM_BYTES, stream>>>(prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ra_bwd_dkdv_kernel<D><<<grid_for(prm.units_kv), NUM_THREADS, KCfg<D>::SMEM_BYTES, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace bwd
+
+cudaError_t launch_bwd(const BwdParams& prm, int d, int num_sms, int max_ctas,
+                       cudaStream_t stream) {
+  if (d == 128) return bwd::launch_bwd_d<128>(prm, num_sms, max_ctas, stream);
+  return bwd::launch_bwd_d<64>(prm, num_sms, max_ctas, stream);
+}
+
+cudaError_t read_and_clear_bwd_status(unsigned long long* out) {
+  unsigned long long v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, bwd::g_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    e = cudaMemcpyToSymbol(bwd::g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return e;
+  }
+  *out = v;
+  return cudaSuccess;
+}
+
+}  // namespace ra

@@ -42,6 +42,7 @@
 #include "ptx_sm100.cuh"
 #include "ra_internal.h"
 #include "ra_merge_math.cuh"
+#include "ra_sync.cuh"
 #include "ring_attn.h"
 
 namespace ra {
@@ -75,10 +76,6 @@ constexpr float RESCALE_LOG2 = 8.0f;
 #define RA_EMU_PERIOD 0
 #endif
 constexpr int EMU_PERIOD = RA_EMU_PERIOD;
-// Longest single hardware suspension inside one mbarrier try_wait (ns).
-#ifndef RA_WAIT_HINT_NS
-#define RA_WAIT_HINT_NS 1000000u
-#endif
 // Minimax (relative error) cubic for 2^f on [-1/2, 1/2], fitted by
 // csrc/fit_exp2_poly.py (Remez exchange); max relative error 7.5e-5 with
 // float32 Horner evaluation.
@@ -209,42 +206,6 @@ __device__ __forceinline__ int unit_for_round(int k, int G, int c) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-struct Ctl {
-  volatile uint32_t* abort;
-  unsigned long long limit_ns;
-};
-
-__device__ __noinline__ void record_timeout(const Ctl& cx, uint32_t site) {
-  *cx.abort = 1u;
-  const unsigned long long code =
-      (static_cast<unsigned long long>(RA_ERR_TIMEOUT) << 32) | (site << 16) | (blockIdx.x & 0xFFFF);
-  atomicCAS(&g_ra_status, 0ull, code);
-}
-
-// Bounded wait on an mbarrier phase.  Returns false if the kernel is aborting
-// (this wait ran out, or another role's did).
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& cx,
-                                         uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity, RA_WAIT_HINT_NS)) return true;
-    if (*cx.abort) return false;
-    if (globaltimer_ns() - t0 > cx.limit_ns) {
-      record_timeout(cx, site);
-      return false;
-    }
-  }
-}
-
-// Short bounded wait used only while draining after an abort.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > ns) return;
-  }
-}
-
 struct Bars {
   uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, o_done0, o_free0, p_half0, drain;
   __device__ __forceinline__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
@@ -255,13 +216,6 @@ struct Bars {
   __device__ __forceinline__ uint32_t o_free(int w) const { return o_free0 + 8u * w; }
   __device__ __forceinline__ uint32_t p_half(int w) const { return p_half0 + 8u * w; }
 };
-
-// Bounded wait executed by a whole warp; the result is warp-uniform.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Ctl& cx,
-                                          uint32_t site) {
-  const bool ok = wait_bar(bar, parity, cx, site);
-  return __all_sync(0xffffffffu, ok);
-}
 
 // ------------------------------------------------------------------ loader
 // The whole warp runs the control flow, so every address and coordinate is
@@ -854,7 +808,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_fwd_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const Ctl cx{abort_flag, p.wait_limit_ns};
+  const Ctl cx{abort_flag, p.wait_limit_ns, &g_ra_status};
 
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(SOFTMAX_REGS));

@@ -40,7 +40,36 @@ struct FwdParams {
   unsigned debug_flags;
 };
 
+// Parameters of the two backward launches (dQ kernel, then dK/dV kernel).
+// tm_q/tm_do view q and dout as {d, Hq, B*L}, tm_k/tm_v view k and v as
+// {d, Hkv, B*L}, with the forward's box and swizzle.
+struct BwdParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_do;
+  const __nv_bfloat16* out;    // forward output O [B, L, Hq, d]
+  const __nv_bfloat16* dout;   // upstream gradient dO [B, L, Hq, d]
+  const float* lse;            // forward lse [B, Hq, L] (natural log)
+  float* dvec;                 // workspace: D = rowsum(dO * O) [B, Hq, L]
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int B, Hq, Hkv, group;
+  int L, blk_len, n_ring, causal;
+  int tiles_per_blk;
+  int units_dq;                // B * Hq * n_ring * tiles_per_blk
+  int units_kv;                // B * Hkv * n_ring * tiles_per_blk
+  float scale;
+  float scale_log2;
+  unsigned long long wait_limit_ns;
+  unsigned debug_flags;
+};
+
 cudaError_t launch_fwd(const FwdParams& prm, int d, int grid, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdParams& prm, int d, int num_sms, int max_ctas,
+                       cudaStream_t stream);
+cudaError_t read_and_clear_bwd_status(unsigned long long* out);
 cudaError_t read_and_clear_status(unsigned long long* out);
 
 cudaError_t launch_merge(const float* o_a, const float* lse_a, const float* o_b,

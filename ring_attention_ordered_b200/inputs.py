@@ -15,6 +15,9 @@ Recipe (identical for every workload):
    a few leading tokens that draw a large share of the attention weight);
 4. round to bf16 with round-to-nearest-even (``Tensor.to(torch.bfloat16)``).
 
+The backward pass's upstream gradient dO is drawn the same way from a
+generator of its own (``make_grad_output``).
+
 The long-context workloads stand in for the pages' Llama-2 / 128K-token runs,
 which need trained weights and datasets that are not used here: the shapes
 (sequence length, heads, head dim, ring size) are the pages', the values are
@@ -125,6 +128,19 @@ def make_inputs(B: int, Hq: int, Hkv: int, L: int, d: int, seed: int,
     k = k.to(torch.bfloat16)
     v = torch.randn((B, L, Hkv, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
     return q, k, v
+
+
+# Seed offset of the upstream gradient dO, so that it is drawn from a
+# generator of its own and never coincides with Q, K or V.
+GRAD_SEED_OFFSET = 1_000_003
+
+
+def make_grad_output(B: int, L: int, Hq: int, d: int, seed: int):
+    """The upstream gradient dO of a backward test or benchmark: standard
+    normal fp32 [B, L, Hq, d] from ``torch.Generator("cpu")`` seeded with
+    ``seed + GRAD_SEED_OFFSET``, rounded to bf16 (nearest even)."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed) + GRAD_SEED_OFFSET)
+    return torch.randn((B, L, Hq, d), generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
 def workload_inputs(w: Workload):

@@ -63,3 +63,38 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what: str = ""):
     assert stats["o_mean"] <= O_MEAN, f"{what}: mean |err| {stats['o_mean']:.3e}; {stats}"
     assert stats["lse_max"] <= LSE_MAX, f"{what}: LSE err {stats['lse_max']:.3e}; {stats}"
     return stats
+
+
+# Gradients (fp64 oracle vs the backward kernels: bf16 inputs, P and dS
+# rounded to bf16 before their products, fp32 accumulation, bf16 outputs).
+# Each element carries the bf16 rounding of its own value (2^-9 relative) and
+# of the terms it sums (P and dS, 2^-9 relative each, with partial
+# cancellation in dK and dQ, whose terms sum to zero over keys); measured
+# against the scale of the tensor:
+#   max |err| <= GRAD_MAX * max |ref| + GRAD_ATOL
+#   mean |err| <= GRAD_MEAN * mean |ref| + GRAD_ATOL
+# GRAD_ATOL covers a gradient that is exactly zero by cancellation (one key
+# per row: dS = P (dP - D) with dP and D the same dot product of O(1) unit
+# normal terms, summed in a different order in fp32, ~1e-6 apart).
+GRAD_MAX = 2.0 ** -6
+GRAD_MEAN = 2.0 ** -8
+GRAD_ATOL = 1e-5
+
+
+def compare_grad(g_gpu, g_ref, what: str = ""):
+    """Assert the gradient tolerances above; return error statistics."""
+    g, r = to_np(g_gpu), np.asarray(g_ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite gradient"
+    err = np.abs(g - r)
+    scale_max = float(np.abs(r).max()) if r.size else 0.0
+    scale_mean = float(np.abs(r).mean()) if r.size else 0.0
+    stats = {
+        "max_err": float(err.max()) if err.size else 0.0,
+        "mean_err": float(err.mean()) if err.size else 0.0,
+        "max_ref": scale_max,
+        "mean_ref": scale_mean,
+    }
+    assert stats["max_err"] <= GRAD_MAX * scale_max + GRAD_ATOL, f"{what}: max {stats}"
+    assert stats["mean_err"] <= GRAD_MEAN * scale_mean + GRAD_ATOL, f"{what}: mean {stats}"
+    return stats

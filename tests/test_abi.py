@@ -46,7 +46,7 @@ def test_status_strings_and_version(lib):
                                  "RA_ERR_CUDA", "RA_ERR_TIMEOUT"]):
         assert _lib.status_string(code) == name
     assert _lib.status_string(99) == "RA_ERR_UNKNOWN"
-    assert _lib.ring_attn_version() == 101
+    assert _lib.ring_attn_version() == 102
 
 
 # Fake, never-dereferenced device addresses: validation rejects these calls
@@ -172,3 +172,49 @@ def test_python_binding_raises_on_error(lib):
         _lib.ring_attn_fwd(Q, K, V, O, LSE, 1, 2, 2, 510, 128, 4, 1, 0.1, 0)
     assert ei.value.status == _lib.RA_ERR_INVALID_ARG
     assert "equal blocks" in str(ei.value)
+
+
+DO, DQ, DK, DV, WS = (7 * A * 64, 8 * A * 64, 9 * A * 64, 10 * A * 64, 11 * A * 64)
+
+
+def bwd_status(lib, **kw):
+    args = dict(q=Q, k=K, v=V, out=O, dout=DO, lse=LSE, dq=DQ, dk=DK, dv=DV, ws=WS,
+                ws_bytes=1 << 20, B=1, Hq=2, Hkv=2, L=512, d=128, n_ring=4, causal=1, scale=0.088)
+    args.update(kw)
+    return lib.ring_attn_bwd(args["q"], args["k"], args["v"], args["out"], args["dout"],
+                             args["lse"], args["dq"], args["dk"], args["dv"], args["ws"],
+                             args["ws_bytes"], args["B"], args["Hq"], args["Hkv"], args["L"],
+                             args["d"], args["n_ring"], args["causal"], args["scale"], None)
+
+
+def test_bwd_workspace_size():
+    assert _lib.ring_attn_bwd_workspace_size(2, 8, 8192) == 2 * 8 * 8192 * 4
+    assert _lib.ring_attn_bwd_workspace_size(0, 8, 8192) == 0
+    with pytest.raises(_lib.RingAttnError):
+        _lib.ring_attn_bwd_workspace_size(-1, 8, 8192)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(L=510), _lib.RA_ERR_INVALID_ARG),
+    (dict(n_ring=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(causal=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), _lib.RA_ERR_INVALID_ARG),
+    (dict(d=96), _lib.RA_ERR_UNSUPPORTED),
+    (dict(dout=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(ws=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(ws_bytes=1 * 2 * 512 * 4 - 4), _lib.RA_ERR_INVALID_ARG),   # workspace too small
+    (dict(dq=DQ + 8), _lib.RA_ERR_INVALID_ARG),                       # not 16-byte aligned
+    (dict(dk=Q + 64), _lib.RA_ERR_INVALID_ARG),                       # dk overlaps q
+    (dict(ws=DV + 64), _lib.RA_ERR_INVALID_ARG),                      # workspace overlaps dv
+    (dict(dv=LSE), _lib.RA_ERR_INVALID_ARG),                          # dv overlaps lse
+])
+def test_bwd_rejects_invalid_arguments(lib, kw, status):
+    assert bwd_status(lib, **kw) == status
+    assert _lib.last_error()
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(L=0), dict(Hq=0, Hkv=0)])
+def test_bwd_empty_problem_launches_nothing(lib, kw):
+    assert bwd_status(lib, q=0, k=0, v=0, out=0, dout=0, lse=0, dq=0, dk=0, dv=0, ws=0,
+                      ws_bytes=0, **kw) == _lib.RA_OK

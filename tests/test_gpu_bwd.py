@@ -1,0 +1,150 @@
+"""GPU parity of the backward pass (ring_attn_bwd, through the C ABI) against
+the fp64 oracle's gradients of the same definition."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import compare_grad
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ra():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from ring_attention_ordered_b200 import _lib, api
+    _lib.load()
+    return api
+
+
+def fwd_bwd(api, q, k, v, do, n_ring, causal, scale=None):
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    out, lse = api.fwd(qd, kd, vd, n_ring, causal, scale)
+    dq, dk, dv = api.bwd(qd, kd, vd, out, dod, lse, n_ring, causal, scale)
+    api.check_status()
+    return dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def full_check(api, B, Hq, Hkv, L, d, n_ring, causal, seed, what):
+    from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
+    q, k, v = make_inputs(B, Hq, Hkv, L, d, seed=seed)
+    do = make_grad_output(B, L, Hq, d, seed=seed)
+    scale = 1.0 / d ** 0.5
+    got = fwd_bwd(api, q, k, v, do, n_ring, causal, scale)
+    ref = oracle.attention_bwd(q, k, v, do, causal, scale)
+    return [compare_grad(g, r, f"{what} {name}") for g, r, name in zip(got, ref, "qkv")]
+
+
+# (B, Hq, Hkv, L, d, n_ring, causal): several tiles, ragged blocks, GQA with
+# even and odd groups, ring sizes 1..5, a single-row sequence
+SMALL = [
+    (1, 1, 1, 128, 128, 1, True),
+    (1, 2, 2, 256, 128, 2, True),
+    (1, 2, 2, 256, 128, 2, False),
+    (2, 4, 2, 384, 64, 3, True),
+    (1, 4, 1, 600, 128, 3, True),      # blocks of 200 rows: a full tile + 72
+    (1, 2, 2, 200, 64, 5, False),      # blocks of 40 rows
+    (1, 3, 1, 512, 128, 4, True),      # group of 3
+    (1, 2, 2, 1024, 128, 4, True),
+    (1, 1, 1, 1, 64, 1, True),         # one row
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d,n_ring,causal", SMALL)
+def test_bwd_small_shapes(ra, B, Hq, Hkv, L, d, n_ring, causal):
+    full_check(ra, B, Hq, Hkv, L, d, n_ring, causal, seed=7 * L + d + n_ring,
+               what=f"{(B, Hq, Hkv, L, d, n_ring, causal)}")
+
+
+def test_bwd_workload_l512_d64_noncausal(ra):
+    full_check(ra, 1, 1, 1, 512, 64, 4, False, seed=0, what="l512")
+
+
+def test_bwd_workload_l8k_h8_causal(ra):
+    """The 8K-token causal workload (B 2, 8 heads, d 128, 4 ring blocks):
+    every gradient element against the oracle."""
+    from ring_attention_ordered_b200.inputs import WORKLOADS
+    w = WORKLOADS["l8k_h8_causal"]
+    full_check(ra, w.B, w.Hq, w.Hkv, w.L, w.d, w.n_ring, w.causal, seed=w.seed, what=w.name)
+
+
+def test_bwd_gqa_workload_dq_rows_and_one_kv_head(ra):
+    """The 32K-token GQA workload (32 query heads on 8 K/V heads, keys x2):
+    sampled dQ rows plus rows around every ring-block boundary, and dK/dV
+    rows of K/V head 0 around the block boundaries (each needs every score
+    row of the group's four heads)."""
+    from ring_attention_ordered_b200.inputs import WORKLOADS, make_grad_output, sample_rows, workload_inputs
+    w = WORKLOADS["l32k_gqa4_causal"]
+    q, k, v = workload_inputs(w)
+    do = make_grad_output(w.B, w.L, w.Hq, w.d, w.seed)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    out, lse = ra.fwd(qd, kd, vd, w.n_ring, w.causal, w.scale)
+    dq, dk, dv = ra.bwd(qd, kd, vd, out, dod, lse, w.n_ring, w.causal, w.scale)
+    ra.check_status()
+    del qd, kd, vd, dod, out, lse
+    lb = w.block_len
+    edges = sorted({r for i in range(w.n_ring + 1) for r in (i * lb - 1, i * lb, i * lb + 127)
+                    if 0 <= r < w.L})
+    bhr = np.concatenate([sample_rows(w, 512),
+                          np.array([[0, h, r] for h in (0, w.Hq - 1) for r in edges], np.int64)])
+    ref = oracle.attention_bwd_dq_rows(q, k, v, do, w.causal, w.scale, bhr)
+    b, h, r = (torch.from_numpy(bhr[:, i]).cuda() for i in range(3))
+    compare_grad(dq[b, r, h, :], ref, "l32k dQ rows")
+    bhc = np.array([[0, 0, r] for r in edges], np.int64)
+    rk, rv = oracle.attention_bwd_kv_rows(q, k, v, do, w.causal, w.scale, bhc)
+    c = torch.from_numpy(bhc[:, 2]).cuda()
+    compare_grad(dk[0, c, 0, :], rk, "l32k dK rows")
+    compare_grad(dv[0, c, 0, :], rv, "l32k dV rows")
+
+
+def test_bwd_deterministic_and_grid_invariant(ra):
+    """Every gradient element is accumulated by one CTA in a fixed order, so
+    the result is bitwise the same whatever the number of CTAs."""
+    from ring_attention_ordered_b200 import _lib
+    from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
+    q, k, v = make_inputs(2, 4, 2, 1024, 128, seed=21)
+    do = make_grad_output(2, 1024, 4, 128, seed=21)
+    ref = fwd_bwd(ra, q, k, v, do, 4, True)
+    try:
+        for cap in (1, 5, 0):
+            _lib.ring_attn_set_max_ctas(cap)
+            got = fwd_bwd(ra, q, k, v, do, 4, True)
+            for a, b in zip(got, ref):
+                assert torch.equal(a, b), cap
+    finally:
+        _lib.ring_attn_set_max_ctas(0)
+
+
+def test_bwd_bounded_wait_reports_timeout_and_recovers(ra):
+    from ring_attention_ordered_b200 import _lib
+    from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
+    q, k, v = (t.cuda() for t in make_inputs(1, 2, 2, 512, 128, seed=22))
+    do = make_grad_output(1, 512, 2, 128, seed=22).cuda()
+    out, lse = ra.fwd(q, k, v, 4, True)
+    ra.check_status()
+    try:
+        _lib.ring_attn_set_wait_limit_ns(200_000_000)
+        _lib.ring_attn_debug_inject(1)
+        ra.bwd(q, k, v, out, do, lse, 4, True)
+        with pytest.raises(_lib.RingAttnError) as ei:
+            ra.check_status()
+        assert ei.value.status == _lib.RA_ERR_TIMEOUT
+    finally:
+        _lib.ring_attn_debug_inject(0)
+        _lib.ring_attn_set_wait_limit_ns(0)
+    full_check(ra, 1, 2, 2, 512, 128, 4, True, seed=22, what="after timeout")
+
+
+def test_bwd_short_workspace_is_rejected(ra):
+    from ring_attention_ordered_b200 import _lib
+    q = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 2, 256), dtype=torch.float32, device="cuda")
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(_lib.RingAttnError) as ei:
+        ra.bwd(q, q.clone(), q.clone(), q.clone(), q.clone(), lse, 2, True, workspace=ws)
+    assert ei.value.status == _lib.RA_ERR_INVALID_ARG
