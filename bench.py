@@ -355,6 +355,43 @@ def run_ours(args, w, world, rank, local):
     merge_bytes = 3 * (4 * w.d + 4) * rows
     del o_a, o_b, l_a, l_b, o_o, l_o
 
+    # the backward pass on the same workload (not part of the timed forward
+    # step): dQ kernel + dK/dV kernel per call, seeded synthetic dO
+    bwd = None
+    if not args.no_bwd:
+        from ring_attention_ordered_b200.inputs import make_grad_output
+        do = make_grad_output(w.B, w.L, w.Hq, w.d, w.seed).to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(16, _lib.ring_attn_bwd_workspace_size(w.B, w.Hq, w.L)),
+                         dtype=torch.uint8, device=dev)
+        api.fwd(q, k, v, w.n_ring, w.causal, w.scale, out=out, lse=lse, stream=stream)
+
+        def bwd_call():
+            api.bwd(q, k, v, out, do, lse, w.n_ring, w.causal, w.scale, dq, dk, dv, ws,
+                    stream=stream)
+
+        for _ in range(2):
+            bwd_call()
+        api.check_status(stream)
+        bsteps = max(2, min(args.steps, 5))
+        if world > 1:
+            dist.barrier()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(bsteps):
+            bwd_call()
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        api.check_status(stream)
+        bwd_ms = max_over_ranks(b0.elapsed_time(b1), world, dev) / bsteps
+        bflops = 2.5 * flops
+        bwd = {"ms": bwd_ms, "TFLOP/s": world * bflops / (bwd_ms / 1e3) / 1e12,
+               "frac_of_burst": bflops / (bwd_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+               "steps": bsteps, "launches_per_call": 2,
+               "flop_convention": "2.5 x forward (five L^2 d products); the two kernels "
+                                  "execute 3.5 x forward (S and dP are recomputed for dQ)"}
+        del do, dq, dk, dv, ws
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -401,6 +438,7 @@ def run_ours(args, w, world, rank, local):
                 "mode": "pipelined: step k+1 copies in and step k-1 copies out while step k computes"},
         "gpu_launches": args.steps,
         "clocks": clocks,
+        "bwd": bwd,
         "merge": {"ms": merge_ms, "GB/s": merge_bytes / (merge_ms / 1e3) / 1e9,
                   "frac_hbm": merge_bytes / (merge_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                   "rows": rows, "d": w.d},
@@ -451,8 +489,67 @@ def run_all_workloads(args):
             "frac_of_burst": tflops / peaks["bf16_tflops"],
             "frac_of_sustained": tflops / peaks["bf16_tflops_sustained"],
             "clocks": clocks}), flush=True)
-        del q, k, v, out, lse
+        from ring_attention_ordered_b200.inputs import make_grad_output
+        do = make_grad_output(w.B, w.L, w.Hq, w.d, w.seed).to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(16, _lib.ring_attn_bwd_workspace_size(w.B, w.Hq, w.L)),
+                         dtype=torch.uint8, device=dev)
+        bsteps = max(1, steps // 2)
+        for _ in range(2):
+            api.bwd(q, k, v, out, do, lse, w.n_ring, w.causal, w.scale, dq, dk, dv, ws, stream=stream)
+        api.check_status(stream)
+        e0.record(stream)
+        for _ in range(bsteps):
+            api.bwd(q, k, v, out, do, lse, w.n_ring, w.causal, w.scale, dq, dk, dv, ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        api.check_status(stream)
+        bms = e0.elapsed_time(e1) / bsteps
+        btf = 2.5 * w.flops() / (bms / 1e3) / 1e12
+        print(json.dumps({
+            "kind": "workload_bwd", "workload": w.describe(), "name": name, "steps": bsteps,
+            "ms": bms, "TFLOP/s": btf, "frac_of_burst": btf / peaks["bf16_tflops"],
+            "flop_convention": "2.5 x forward"}), flush=True)
+        del q, k, v, out, lse, do, dq, dk, dv, ws
         torch.cuda.empty_cache()
+    return 0
+
+
+def run_bwd_only(args, w):
+    """The backward pass alone on one workload (not the contract line): one
+    forward, W warm-up and K timed ring_attn_bwd calls; one JSON line."""
+    import torch
+
+    from ring_attention_ordered_b200 import _lib, api
+    from ring_attention_ordered_b200.inputs import make_grad_output, workload_inputs
+
+    _lib.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    q, k, v = (t.to(dev) for t in workload_inputs(w))
+    do = make_grad_output(w.B, w.L, w.Hq, w.d, w.seed).to(dev)
+    out, lse = api.fwd(q, k, v, w.n_ring, w.causal, w.scale, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(16, _lib.ring_attn_bwd_workspace_size(w.B, w.Hq, w.L)),
+                     dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        api.bwd(q, k, v, out, do, lse, w.n_ring, w.causal, w.scale, dq, dk, dv, ws, stream=stream)
+    api.check_status(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        api.bwd(q, k, v, out, do, lse, w.n_ring, w.causal, w.scale, dq, dk, dv, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    api.check_status(stream)
+    ms = e0.elapsed_time(e1) / max(1, args.steps)
+    tf = 2.5 * w.flops() / (ms / 1e3) / 1e12
+    print(json.dumps({"kind": "bwd", "workload": w.describe(), "name": w.name,
+                      "steps": args.steps, "warmup": args.warmup, "ms": ms, "TFLOP/s": tf,
+                      "frac_of_burst": tf / peaks["bf16_tflops"],
+                      "flop_convention": "2.5 x forward"}), flush=True)
     return 0
 
 
@@ -532,9 +629,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass leg")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--all-workloads", action="store_true",
                     help="print one line per named workload instead of the benchmark line")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="time only the backward pass on the workload")
     ap.add_argument("--ring-emulated", action="store_true",
                     help="time every host of the multi-host ring on this GPU (three layouts)")
     ap.add_argument("--ref-budget", type=float, default=None,
@@ -551,6 +651,8 @@ def main():
         return run_all_workloads(args)
     if args.ring_emulated:
         return run_ring_emulated(args, w)
+    if args.bwd_only:
+        return run_bwd_only(args, w)
     return run_ours(args, w, world, rank, local)
 
 
