@@ -170,6 +170,39 @@ ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void*
                         ra_stream_t stream);
 
 /*
+ * ring_attn_bwd_noalloc -- ring_attn_bwd for callers that cannot allocate
+ * device memory for its workspace.  The pages have no counterpart: this is
+ * an interface convenience, not a step of the method.
+ *
+ * Who needs it: a caller whose device memory is owned by someone else (a
+ * framework's caching allocator or a fixed budget reserved at start-up that
+ * this library cannot draw from), or one that must not call cudaMalloc and
+ * cudaFree on its hot path because cudaFree synchronises the device.  This
+ * entry point allocates nothing: the D vector that ring_attn_bwd keeps in the
+ * caller's workspace lives here in a fixed device array of the library
+ * (4 MiB: B * Hq * L <= 1,048,576 query rows), which is part of the loaded
+ * module rather than created by any allocation call.
+ *
+ *   Arguments, layouts, results and errors: those of ring_attn_bwd without
+ *   the workspace pair; the results are bitwise those of ring_attn_bwd.
+ *   B * Hq * L above 1,048,576 is rejected with RA_ERR_INVALID_ARG before
+ *   anything is launched (use ring_attn_bwd with a workspace instead).
+ *
+ * Nothing in the fixed array has to start at zero: each call writes every
+ * entry it later reads.  The array is shared by every call on a device, so
+ * two calls whose kernels may run at the same time (on different streams,
+ * or from different host threads) race on it and corrupt each other's
+ * results: order them on one stream, or use ring_attn_bwd with a workspace
+ * per concurrent call.  The first call on each device looks up the array's
+ * address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture begins.
+ */
+ra_status ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                int B, int Hq, int Hkv, int64_t L, int d, int n_ring, int causal,
+                                float scale, ra_stream_t stream);
+
+/*
  * ring_attn_merge -- fold two partial attention results over disjoint key
  * sets into one (the accumulation of each ring step's blockwise result into
  * O_i, "Ring Attention 环注意力" L4 §4.2 step 2, kept as output plus

@@ -10,6 +10,7 @@ and the seeded synthetic inputs (``inputs``).
 from ._lib import (  # noqa: F401
     RingAttnError,
     ring_attn_bwd,
+    ring_attn_bwd_noalloc,
     ring_attn_bwd_workspace_size,
     ring_attn_check_status,
     ring_attn_debug_inject,

@@ -28,6 +28,8 @@ SIGNATURES = {
     "ring_attn_bwd_workspace_size": (_I, [_I, _I, _I64, ctypes.POINTER(ctypes.c_size_t)]),
     "ring_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I64,
                            _I, _I, _I, ctypes.c_float, _P]),
+    "ring_attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I,
+                                   ctypes.c_float, _P]),
     "ring_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I, _P]),
     "ring_attn_check_status": (_I, [_P]),
     "ring_attn_set_wait_limit_ns": (_I, [ctypes.c_uint64]),
@@ -95,6 +97,13 @@ def ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace, workspace_byte
     return _check(load().ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace,
                                        workspace_bytes, B, Hq, Hkv, L, d, n_ring,
                                        int(bool(causal)), float(scale), stream))
+
+
+def ring_attn_bwd_noalloc(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, L, d, n_ring, causal,
+                          scale, stream=0):
+    return _check(load().ring_attn_bwd_noalloc(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv,
+                                               L, d, n_ring, int(bool(causal)), float(scale),
+                                               stream))
 
 
 def ring_attn_fwd_visit(q, k, v, o_acc, lse_acc, out, B, Hq, Hkv, l, d, diag, fold, scale,

@@ -93,6 +93,29 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
     return dq, dk, dv
 
 
+def bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                dout: torch.Tensor, lse: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor,
+                dv: torch.Tensor, n_ring: int, causal: bool, scale: float | None = None,
+                stream=None):
+    """``bwd`` through ring_attn_bwd_noalloc: no workspace, results written
+    into the given dq/dk/dv (bf16, shapes of q/k/v); B * Hq * L must not
+    exceed 1,048,576."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"),
+                 (dk, "dk"), (dv, "dv")):
+        _check_cuda(t, n, torch.bfloat16, 4)
+    _check_cuda(lse, "lse", torch.float32, 3)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(q.device):
+        _lib.ring_attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                   dv.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale,
+                                   _stream_handle(stream))
+    return dq, dk, dv
+
+
 def fwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Tensor,
               lse_acc: torch.Tensor, diag: int, fold: bool, scale: float | None = None,
               out: torch.Tensor | None = None, stream=None):

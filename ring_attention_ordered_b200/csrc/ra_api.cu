@@ -317,6 +317,31 @@ ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void*
   return ok();
 }
 
+ra_status ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                int B, int Hq, int Hkv, int64_t L, int d, int n_ring, int causal,
+                                float scale, ra_stream_t stream) {
+  if (B < 0 || Hq < 0 || L < 0)
+    return fail(RA_ERR_INVALID_ARG, "negative size (B=%d Hq=%d L=%lld)", B, Hq,
+                static_cast<long long>(L));
+  const long long rows = static_cast<long long>(B) * Hq * L;
+  if (rows > ra::kNoAllocScratchRows)
+    return fail(RA_ERR_INVALID_ARG,
+                "B*Hq*L = %lld query rows exceed the %lld rows (%lld bytes) of static scratch "
+                "of ring_attn_bwd_noalloc; use ring_attn_bwd with a workspace",
+                rows, ra::kNoAllocScratchRows, ra::kNoAllocScratchRows * 4);
+  if (rows == 0)
+    return ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, nullptr, 0, B, Hq, Hkv, L, d,
+                         n_ring, causal, scale, stream);
+  void* scratch = nullptr;
+  cudaError_t e = ra::noalloc_scratch(&scratch);
+  if (e != cudaSuccess)
+    return fail(RA_ERR_CUDA, "static scratch lookup: %s", cudaGetErrorString(e));
+  return ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, scratch,
+                       static_cast<size_t>(ra::kNoAllocScratchRows) * 4, B, Hq, Hkv, L, d, n_ring,
+                       causal, scale, stream);
+}
+
 ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b,
                           const float* lse_b, float* o_out, float* lse_out, int64_t rows, int d,
                           ra_stream_t stream) {

@@ -35,6 +35,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "ptx_sm100.cuh"
 #include "ra_internal.h"
@@ -951,6 +952,28 @@ cudaError_t launch_bwd(const BwdParams& prm, int d, int num_sms, int max_ctas,
                        cudaStream_t stream) {
   if (d == 128) return bwd::launch_bwd_d<128>(prm, num_sms, max_ctas, stream);
   return bwd::launch_bwd_d<64>(prm, num_sms, max_ctas, stream);
+}
+
+// Fixed device scratch for ring_attn_bwd_noalloc: one fp32 D value per query
+// row and head, for problems with B * Hq * L <= kNoAllocScratchRows.  It is
+// part of the module image (no allocation call creates it); every call
+// overwrites the entries it reads, so nothing in it has to start at zero.
+__device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchRows];
+
+cudaError_t noalloc_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    e = cudaGetSymbolAddress(&addr[dev], g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }
 
 cudaError_t read_and_clear_bwd_status(unsigned long long* out) {

@@ -70,6 +70,11 @@ cudaError_t launch_fwd(const FwdParams& prm, int d, int grid, cudaStream_t strea
 cudaError_t launch_bwd(const BwdParams& prm, int d, int num_sms, int max_ctas,
                        cudaStream_t stream);
 cudaError_t read_and_clear_bwd_status(unsigned long long* out);
+
+// Static scratch of ring_attn_bwd_noalloc (fp32 entries, 4 MiB).
+constexpr long long kNoAllocScratchRows = 1ll << 20;
+// Address of that scratch on the current device (looked up once per device).
+cudaError_t noalloc_scratch(void** ptr);
 cudaError_t read_and_clear_status(unsigned long long* out);
 
 cudaError_t launch_merge(const float* o_a, const float* lse_a, const float* o_b,
