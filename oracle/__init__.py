@@ -44,4 +44,5 @@ from .attn_bwd_fp64 import (  # noqa: F401
     attention_bwd,
     attention_bwd_dq_rows,
     attention_bwd_kv_rows,
+    block_attention_bwd,
 )

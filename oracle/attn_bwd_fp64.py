@@ -18,9 +18,12 @@ gradient dO:
 
 With grouped-query attention (lnwmold §2.2, contiguous groups) a K/V head's
 gradient is the sum over the query heads of its group.  Masked entries of A
-are exactly zero and contribute nothing.  Everything here is written from
-that definition; no identity the kernels use (such as rowsum(A * dA) =
-rowsum(dO * O)) is assumed.
+are exactly zero and contribute nothing.  ``attention_bwd`` and the row
+functions are written from that definition and use no identity the kernels
+use.  ``block_attention_bwd`` (one ring visit's share) cannot see the other
+blocks' weights, so it writes the Jacobian's row term through the forward
+output, rowsum(A * dA) = rowsum(dO * O); it is pinned by summing its shares
+over all visits back to ``attention_bwd``.
 """
 
 from __future__ import annotations
@@ -122,3 +125,51 @@ def attention_bwd_kv_rows(q, k, v, dout, causal: bool, scale: float, bhc, row_bl
                 dv[idx] += a[:, cs].T @ dh[r0:r1]
                 dk[idx] += scale * (ds[:, cs].T @ qh[r0:r1])
     return dk, dv
+
+
+def block_attention_bwd(q, k, v, out, dout, lse, scale: float, kind: str):
+    """One ring visit's share of the gradients: the query block (rows r, with
+    their forward output ``out`` and natural-log ``lse`` over the WHOLE
+    sequence) against one K/V block under the visit mask ``kind`` of
+    ``attn_fp64.block_attention`` ("full", "masked" keys c <= r, "strict"
+    keys c < r).  With A the rows' attention weights restricted to this
+    block's keys (A = exp(scale q.k - lse), the block's columns of the full
+    softmax) and the Jacobian's row term rowsum(A_full * dA_full) written as
+    rowsum(dO * O) (O = A_full V):
+
+        dV_part = A^T dO,   dS = A * (dO V^T - rowsum(dO * O))
+        dQ_part = scale dS K,   dK_part = scale dS^T Q
+
+    Summed over every K/V block a query block visits, the parts are the
+    gradients of :func:`attention_bwd` (the pin of this function).
+    q, out, dout [B, lq, Hq, d]; k, v [B, lk, Hkv, d]; lse [B, Hq, lq].
+    Returns float64 (dq_part, dk_part, dv_part)."""
+    q, k, v, o, do, lse = (_f64(x) for x in (q, k, v, out, dout, lse))
+    B, lq, Hq, d = q.shape
+    lk, Hkv = k.shape[1], k.shape[2]
+    if kind not in ("full", "masked", "strict"):
+        raise ValueError(f"unknown visit kind {kind!r}")
+    if kind != "full" and lq != lk:
+        raise ValueError("masked visits need equal block lengths")
+    g = Hq // Hkv
+    rows = np.arange(lq)[:, None]
+    cols = np.arange(lk)[None, :]
+    allowed = np.ones((lq, lk), dtype=bool)
+    if kind == "masked":
+        allowed = cols <= rows
+    elif kind == "strict":
+        allowed = cols < rows
+    dq = np.zeros((B, lq, Hq, d))
+    dk = np.zeros((B, lk, Hkv, d))
+    dv = np.zeros((B, lk, Hkv, d))
+    for b in range(B):
+        for h in range(Hq):
+            kh = h // g
+            s = scale * (q[b, :, h, :] @ k[b, :, kh, :].T)
+            a = np.where(allowed, np.exp(s - lse[b, h][:, None]), 0.0)
+            rterm = (do[b, :, h, :] * o[b, :, h, :]).sum(axis=1, keepdims=True)
+            ds = a * (do[b, :, h, :] @ v[b, :, kh, :].T - rterm)
+            dv[b, :, kh, :] += a.T @ do[b, :, h, :]
+            dq[b, :, h, :] = scale * (ds @ k[b, :, kh, :])
+            dk[b, :, kh, :] += scale * (ds.T @ q[b, :, h, :])
+    return dq, dk, dv

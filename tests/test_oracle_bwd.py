@@ -188,3 +188,61 @@ def test_clean_bwd_mutant_template_passes():
     for pin in BWD_PINS:
         pin(_mutant(None))
     assert ob.attention_bwd is oracle.attention_bwd
+
+
+# --------------------------------------------------------------------------
+# block_attention_bwd: one ring visit's share of the gradients
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n_blocks", [1, 2, 4])
+def test_block_bwd_parts_sum_to_the_gradient(causal, n_blocks):
+    """With the forward oracle's own output and lse, the parts of every
+    (query block, key block) pair the mask allows -- diagonal blocks
+    "masked", earlier blocks "full" -- add up to attention_bwd."""
+    q, k, v, do = problem(6, B=2, L=24, Hq=4, Hkv=2, d=5)
+    scale = 0.45
+    out, lse = oa.attention(q, k, v, causal, scale)
+    want = oracle.attention_bwd(q, k, v, do, causal, scale)
+    lb = 24 // n_blocks
+    got = [np.zeros_like(x) for x in (q, k, v)]
+    for i in range(n_blocks):
+        rq = slice(i * lb, (i + 1) * lb)
+        for j in range(n_blocks):
+            if causal and j > i:
+                continue
+            rk = slice(j * lb, (j + 1) * lb)
+            kind = "masked" if (causal and i == j) else "full"
+            pq, pk, pv = oracle.block_attention_bwd(q[:, rq], k[:, rk], v[:, rk], out[:, rq],
+                                                    do[:, rq], lse[:, :, rq], scale, kind)
+            got[0][:, rq] += pq
+            got[1][:, rk] += pk
+            got[2][:, rk] += pv
+    for g_, w_ in zip(got, want):
+        np.testing.assert_allclose(g_, w_, rtol=0, atol=1e-12)
+
+
+def test_block_bwd_strict_is_the_shifted_masked_visit():
+    """Keys c < r: row 0 receives nothing and key L-1 gives nothing; the
+    strict visit equals the masked visit minus the diagonal pairs, checked
+    by adding the diagonal's share, formed from the definition one pair at a
+    time with math.fsum."""
+    import math
+    q, k, v, do = problem(7, B=1, L=6, Hq=2, Hkv=1, d=3)
+    scale = 0.8
+    out, lse = oa.attention(q, k, v, True, scale)
+    sq, sk, sv = oracle.block_attention_bwd(q, k, v, out, do, lse, scale, "strict")
+    mq, mk, mv = oracle.block_attention_bwd(q, k, v, out, do, lse, scale, "masked")
+    assert np.all(sq[:, 0] == 0.0)
+    dq_d, dk_d, dv_d = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for h in range(2):
+        for r in range(6):
+            a = math.exp(scale * math.fsum(q[0, r, h] * k[0, r, 0]) - lse[0, h, r])
+            da = math.fsum(do[0, r, h] * v[0, r, 0])
+            rt = math.fsum(do[0, r, h] * out[0, r, h])
+            ds = a * (da - rt)
+            dv_d[0, r, 0] += a * do[0, r, h]
+            dq_d[0, r, h] += scale * ds * k[0, r, 0]
+            dk_d[0, r, 0] += scale * ds * q[0, r, h]
+    for s_, m_, d_ in ((sq, mq, dq_d), (sk, mk, dk_d), (sv, mv, dv_d)):
+        np.testing.assert_allclose(s_ + d_, m_, rtol=0, atol=1e-12)
