@@ -170,6 +170,55 @@ ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void*
                         ra_stream_t stream);
 
 /*
+ * ring_attn_bwd_visit -- one ring step of the backward pass on one host: its
+ * query block against the K/V block it holds, adding the step's share to the
+ * host's dQ accumulator and to the travelling dK, dV accumulators of that
+ * K/V block (which move around the ring with K and V, as in "Ring Attention
+ * 环注意力" L4 §4.2, so that every host adds its share before the block
+ * returns home).  The arithmetic is ring_attn_bwd's, restricted to one
+ * (query block, K/V block) pair with the mask `diag` of ring_attn_fwd_visit
+ * (0 every key, 1 keys c <= r, 2 keys c < r; local rows):
+ *
+ *   parts & 1: D = rowsum(dout * out) of the query block into `workspace`,
+ *              then dq_acc (fp32 [B, l, Hq, d]) = (fold_q ? dq_acc : 0)
+ *              + scale * dS K; dq (bf16, may be NULL) gets the rounded
+ *              new dq_acc.
+ *   parts & 2: dk_acc, dv_acc (fp32 [B, l, Hkv, d]) = (fold_kv ? acc : 0)
+ *              + scale * dS^T Q, P^T dO; reads D from `workspace`, which an
+ *              earlier call with parts & 1 for the same query block (out,
+ *              dout) must have written on the same stream.
+ *   Both halves may be launched by one call (parts = 3), or separately so
+ *   that a caller can receive the incoming dK, dV accumulators while the dQ
+ *   half computes.
+ *
+ *   q, out, dout  bf16 [B, l, Hq, d]: the host's query block, its forward
+ *                 output and the loss gradient for it                 (in)
+ *   lse           fp32 [B, Hq, l]: the host's final forward lse (over the
+ *                 whole sequence, not this visit)                     (in)
+ *   k, v          bf16 [B, l, Hkv, d]: the visited K/V block            (in)
+ *   workspace     >= B * Hq * l * 4 bytes (ring_attn_bwd_workspace_size
+ *                 with L = l)                                        (in/out)
+ *   B, Hq, Hkv, l, d, scale   as for ring_attn_fwd with L = l, n_ring = 1;
+ *   diag 0..2; parts 1..3; fold_q, fold_kv 0 or 1.
+ *
+ * Pointers must be 16-byte aligned; accumulators, dq and workspace must not
+ * overlap the inputs or each other.  Errors as for ring_attn_bwd.
+ */
+ra_status ring_attn_bwd_visit(const void* q, const void* k, const void* v, const void* out,
+                              const void* dout, const float* lse, float* dq_acc, float* dk_acc,
+                              float* dv_acc, void* dq, void* workspace, size_t workspace_bytes,
+                              int B, int Hq, int Hkv, int64_t l, int d, int diag, int parts,
+                              int fold_q, int fold_kv, float scale, ra_stream_t stream);
+
+/*
+ * ring_attn_round_bf16 -- dst[i] = src[i] rounded to bf16 (nearest even),
+ * i < n: turns a travelling fp32 gradient accumulator into the bf16 result
+ * once it is home.  src fp32, dst bf16, both 16-byte aligned, n % 8 == 0,
+ * no overlap.  n == 0 launches nothing.
+ */
+ra_status ring_attn_round_bf16(const float* src, void* dst, int64_t n, ra_stream_t stream);
+
+/*
  * ring_attn_bwd_noalloc -- ring_attn_bwd for callers that cannot allocate
  * device memory for its workspace.  The pages have no counterpart: this is
  * an interface convenience, not a step of the method.

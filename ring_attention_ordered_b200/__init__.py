@@ -11,12 +11,14 @@ from ._lib import (  # noqa: F401
     RingAttnError,
     ring_attn_bwd,
     ring_attn_bwd_noalloc,
+    ring_attn_bwd_visit,
     ring_attn_bwd_workspace_size,
     ring_attn_check_status,
     ring_attn_debug_inject,
     ring_attn_fwd,
     ring_attn_fwd_visit,
     ring_attn_merge,
+    ring_attn_round_bf16,
     ring_attn_set_max_ctas,
     ring_attn_set_schedule,
     ring_attn_set_wait_limit_ns,

@@ -28,6 +28,9 @@ SIGNATURES = {
     "ring_attn_bwd_workspace_size": (_I, [_I, _I, _I64, ctypes.POINTER(ctypes.c_size_t)]),
     "ring_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I64,
                            _I, _I, _I, ctypes.c_float, _P]),
+    "ring_attn_bwd_visit": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I,
+                                 _I, _I64, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    "ring_attn_round_bf16": (_I, [_P, _P, _I64, _P]),
     "ring_attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I,
                                    ctypes.c_float, _P]),
     "ring_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I, _P]),
@@ -97,6 +100,19 @@ def ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace, workspace_byte
     return _check(load().ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace,
                                        workspace_bytes, B, Hq, Hkv, L, d, n_ring,
                                        int(bool(causal)), float(scale), stream))
+
+
+def ring_attn_bwd_visit(q, k, v, out, dout, lse, dq_acc, dk_acc, dv_acc, dq, workspace,
+                        workspace_bytes, B, Hq, Hkv, l, d, diag, parts, fold_q, fold_kv, scale,
+                        stream=0):
+    return _check(load().ring_attn_bwd_visit(q, k, v, out, dout, lse, dq_acc, dk_acc, dv_acc, dq,
+                                             workspace, workspace_bytes, B, Hq, Hkv, l, d,
+                                             int(diag), int(parts), int(fold_q), int(fold_kv),
+                                             float(scale), stream))
+
+
+def ring_attn_round_bf16(src, dst, n, stream=0):
+    return _check(load().ring_attn_round_bf16(src, dst, n, stream))
 
 
 def ring_attn_bwd_noalloc(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, L, d, n_ring, causal,

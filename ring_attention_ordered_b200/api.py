@@ -116,6 +116,52 @@ def bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
     return dq, dk, dv
 
 
+def bwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+              dout: torch.Tensor, lse: torch.Tensor, workspace: torch.Tensor, diag: int,
+              parts: int, dq_acc: torch.Tensor | None = None, dk_acc: torch.Tensor | None = None,
+              dv_acc: torch.Tensor | None = None, fold_q: bool = False, fold_kv: bool = False,
+              scale: float | None = None, dq: torch.Tensor | None = None, stream=None):
+    """One backward ring visit (ring_attn_bwd_visit): the host's query block
+    q/out/dout [B, l, Hq, d] (bf16) with its final lse [B, Hq, l] against the
+    K/V block k/v [B, l, Hkv, d]; parts 1 (dQ, writes D to workspace), 2
+    (dK/dV, reads D) or 3.  Accumulators are fp32 of the shapes of q and k."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check_cuda(t, n, torch.bfloat16, 4)
+    _check_cuda(lse, "lse", torch.float32, 3)
+    B, l, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, l, Hkv, d) or v.shape != k.shape or out.shape != q.shape or \
+            dout.shape != q.shape or lse.shape != (B, Hq, l):
+        raise ValueError("block shapes do not match")
+    for t, n, ref in ((dq_acc, "dq_acc", q), (dk_acc, "dk_acc", k), (dv_acc, "dv_acc", k)):
+        if t is not None:
+            _check_cuda(t, n, torch.float32, 4)
+            if t.shape != ref.shape:
+                raise ValueError(f"{n} shape does not match")
+    if dq is not None:
+        _check_cuda(dq, "dq", torch.bfloat16, 4)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ptr = lambda t: 0 if t is None else t.data_ptr()  # noqa: E731
+    with torch.cuda.device(q.device):
+        _lib.ring_attn_bwd_visit(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 dout.data_ptr(), lse.data_ptr(), ptr(dq_acc), ptr(dk_acc),
+                                 ptr(dv_acc), ptr(dq), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), B, Hq, Hkv, l, d,
+                                 diag, parts, fold_q, fold_kv, scale, _stream_handle(stream))
+
+
+def round_bf16(src: torch.Tensor, dst: torch.Tensor | None = None, stream=None):
+    """fp32 -> bf16 (nearest even) through ring_attn_round_bf16."""
+    if not src.is_cuda or src.dtype != torch.float32 or not src.is_contiguous():
+        raise TypeError("src must be a contiguous fp32 CUDA tensor")
+    dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device) if dst is None else dst
+    with torch.cuda.device(src.device):
+        _lib.ring_attn_round_bf16(src.data_ptr(), dst.data_ptr(), src.numel(),
+                                  _stream_handle(stream))
+    return dst
+
+
 def fwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Tensor,
               lse_acc: torch.Tensor, diag: int, fold: bool, scale: float | None = None,
               out: torch.Tensor | None = None, stream=None):

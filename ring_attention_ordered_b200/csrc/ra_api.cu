@@ -311,9 +311,111 @@ ra_status ring_attn_bwd(const void* q, const void* k, const void* v, const void*
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.wait_limit_ns = g_wait_limit_ns.load();
   prm.debug_flags = g_debug_flags.load();
+  prm.parts = 3;
   cudaError_t e = ra::launch_bwd(prm, d, sms, g_max_ctas.load(),
                                  reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+ra_status ring_attn_bwd_visit(const void* q, const void* k, const void* v, const void* out,
+                              const void* dout, const float* lse, float* dq_acc, float* dk_acc,
+                              float* dv_acc, void* dq, void* workspace, size_t workspace_bytes,
+                              int B, int Hq, int Hkv, int64_t l, int d, int diag, int parts,
+                              int fold_q, int fold_kv, float scale, ra_stream_t stream) {
+  if (diag < 0 || diag > 2) return fail(RA_ERR_INVALID_ARG, "diag must be 0, 1 or 2");
+  if (parts < 1 || parts > 3) return fail(RA_ERR_INVALID_ARG, "parts must be 1, 2 or 3");
+  if ((fold_q != 0 && fold_q != 1) || (fold_kv != 0 && fold_kv != 1))
+    return fail(RA_ERR_INVALID_ARG, "fold flags must be 0 or 1");
+  ra_status st = check_forward_shape(B, Hq, Hkv, l, d, 1, diag != 0, scale);
+  if (st != RA_OK) return st;
+  if (static_cast<long long>(B) * Hq * l == 0) return ok();
+  const size_t nq = static_cast<size_t>(B) * l * Hq * d * 2;
+  const size_t nkv = static_cast<size_t>(B) * l * Hkv * d * 2;
+  const size_t nl = static_cast<size_t>(B) * Hq * l * 4;
+  if (!q || !k || !v || !out || !dout || !lse || !workspace)
+    return fail(RA_ERR_INVALID_ARG, "null pointer");
+  if ((parts & 1) && !dq_acc) return fail(RA_ERR_INVALID_ARG, "dq_acc is needed for the dQ part");
+  if ((parts & 2) && (!dk_acc || !dv_acc))
+    return fail(RA_ERR_INVALID_ARG, "dk_acc and dv_acc are needed for the dK/dV part");
+  const void* ptrs[11] = {q, k, v, out, dout, lse, workspace, dq_acc, dk_acc, dv_acc, dq};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(RA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (workspace_bytes < nl)
+    return fail(RA_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed",
+                workspace_bytes, nl);
+  const void* ins[6] = {q, k, v, out, dout, lse};
+  const size_t in_n[6] = {nq, nkv, nkv, nq, nq, nl};
+  const void* outs[5] = {workspace, (parts & 1) ? dq_acc : nullptr, (parts & 1) ? dq : nullptr,
+                         (parts & 2) ? dk_acc : nullptr, (parts & 2) ? dv_acc : nullptr};
+  const size_t out_n[5] = {nl, 2 * nq, nq, 2 * nkv, 2 * nkv};
+  for (int o = 0; o < 5; ++o) {
+    if (!outs[o]) continue;
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(outs[o], out_n[o], ins[i], in_n[i]))
+        return fail(RA_ERR_INVALID_ARG, "an output or the workspace overlaps an input");
+    for (int o2 = o + 1; o2 < 5; ++o2)
+      if (outs[o2] && overlaps(outs[o], out_n[o], outs[o2], out_n[o2]))
+        return fail(RA_ERR_INVALID_ARG, "outputs and workspace overlap each other");
+  }
+  int sms = 0;
+  if ((st = device_info(&sms)) != RA_OK) return st;
+  ra::BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const long long rows = static_cast<long long>(B) * l;
+  if ((st = make_map(&prm.tm_q, q, Hq, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_k, k, Hkv, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_v, v, Hkv, rows, d)) != RA_OK) return st;
+  if ((st = make_map(&prm.tm_do, dout, Hq, rows, d)) != RA_OK) return st;
+  prm.out = static_cast<const __nv_bfloat16*>(out);
+  prm.dout = static_cast<const __nv_bfloat16*>(dout);
+  prm.lse = lse;
+  prm.dvec = static_cast<float*>(workspace);
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.L = static_cast<int>(l);
+  prm.n_ring = 1;
+  prm.blk_len = static_cast<int>(l);
+  prm.causal = diag != 0;
+  prm.tiles_per_blk = (prm.blk_len + 127) / 128;
+  const long long uq = static_cast<long long>(B) * Hq * prm.tiles_per_blk;
+  if (uq >= (1ll << 31)) return fail(RA_ERR_INVALID_ARG, "problem too large (%lld work units)", uq);
+  prm.units_dq = static_cast<int>(uq);
+  prm.units_kv = static_cast<int>(static_cast<long long>(B) * Hkv * prm.tiles_per_blk);
+  prm.scale = scale;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.wait_limit_ns = g_wait_limit_ns.load();
+  prm.debug_flags = g_debug_flags.load();
+  prm.parts = parts;
+  prm.dq_acc = dq_acc;
+  prm.dk_acc = dk_acc;
+  prm.dv_acc = dv_acc;
+  prm.fold_q = fold_q;
+  prm.fold_kv = fold_kv;
+  prm.diag_shift = diag == 2;
+  cudaError_t e = ra::launch_bwd(prm, d, sms, g_max_ctas.load(),
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "backward visit launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+ra_status ring_attn_round_bf16(const float* src, void* dst, int64_t n, ra_stream_t stream) {
+  if (n < 0) return fail(RA_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return ok();
+  if (!src || !dst) return fail(RA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(src) || !aligned16(dst) || n % 8 != 0)
+    return fail(RA_ERR_INVALID_ARG, "pointers must be 16-byte aligned and n a multiple of 8");
+  if (overlaps(src, static_cast<size_t>(n) * 4, dst, static_cast<size_t>(n) * 2))
+    return fail(RA_ERR_INVALID_ARG, "dst overlaps src");
+  int sms = 0;
+  ra_status st = device_info(&sms);
+  if (st != RA_OK) return st;
+  cudaError_t e = ra::launch_round_bf16(src, static_cast<__nv_bfloat16*>(dst), n, sms,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "round launch: %s", cudaGetErrorString(e));
   return ok();
 }
 
@@ -424,6 +526,6 @@ const char* ring_attn_status_string(ra_status s) {
 
 const char* ring_attn_last_error(void) { return g_last_error.c_str(); }
 
-int ring_attn_version(void) { return 102; }
+int ring_attn_version(void) { return 103; }
 
 }  // extern "C"

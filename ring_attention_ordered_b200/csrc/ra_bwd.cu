@@ -130,6 +130,50 @@ __device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bf
   }
 }
 
+// Per-visit form of store_acc_row: the row (times `mul`) is written to, or
+// with `fold` added to, the fp32 accumulator row acc (D floats); `dst`, if
+// not null, receives the bf16 rounding of the new accumulator row.
+template <int D>
+__device__ __forceinline__ void fold_acc_row(uint32_t taddr, float mul, float* acc, bool fold,
+                                             __nv_bfloat16* dst, bool valid) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    tmem_ld32(taddr + cc * 32, o);
+    tmem_wait_ld();
+    if (valid) {
+      float4* a4 = reinterpret_cast<float4*>(acc + cc * 32);
+      float r[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 x = make_float4(__uint_as_float(o[4 * j]) * mul, __uint_as_float(o[4 * j + 1]) * mul,
+                               __uint_as_float(o[4 * j + 2]) * mul,
+                               __uint_as_float(o[4 * j + 3]) * mul);
+        if (fold) {
+          const float4 a = a4[j];
+          x.x += a.x;
+          x.y += a.y;
+          x.z += a.z;
+          x.w += a.w;
+        }
+        a4[j] = x;
+        r[4 * j] = x.x;
+        r[4 * j + 1] = x.y;
+        r[4 * j + 2] = x.z;
+        r[4 * j + 3] = x.w;
+      }
+      if (dst != nullptr) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          d4[j] = make_uint4(pack_bf16x2(r[8 * j], r[8 * j + 1]), pack_bf16x2(r[8 * j + 2], r[8 * j + 3]),
+                             pack_bf16x2(r[8 * j + 4], r[8 * j + 5]),
+                             pack_bf16x2(r[8 * j + 6], r[8 * j + 7]));
+      }
+    }
+  }
+}
+
 // dS over 32 columns: ds = p * (dp - D), p from bf16 pairs pk (16 words), dp
 // from TMEM (fp32), D per column (dkdv: one per query, from shared memory)
 // or one for the whole row (dq: the row's own D).
@@ -406,7 +450,7 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, c
     it.start(p, x);
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
       int lim = min(TM, p.blk_len - it.kl * TM) - 1;
-      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * TM);
+      if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * TM - p.diag_shift);
       const bool masked = __any_sync(0xffffffffu, lim < TM - 1);
       if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
       tc_fence_after();
@@ -455,8 +499,11 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, c
     // epilogue: dQ = scale * (dS K) accumulated in TMEM
     if (!wait_warp(br.acc_done(), units & 1u, cx, SITE_ACC_DONE)) return;
     tc_fence_after();
-    __nv_bfloat16* dst = p.dq + ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D;
-    store_acc_row<D>(t_dq, p.scale, dst, valid);
+    const long long qoff = ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D;
+    if (p.dq_acc != nullptr)
+      fold_acc_row<D>(t_dq, p.scale, p.dq_acc + qoff, p.fold_q, p.dq ? p.dq + qoff : nullptr, valid);
+    else
+      store_acc_row<D>(t_dq, p.scale, p.dq + qoff, valid);
     tc_fence_before();
     mbar_arrive(br.acc_free());
     ++units;
@@ -788,7 +835,7 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
       const int s = q_it % C::NS;
       // the diagonal tile of the own block: query column j sees key row t
-      // only when j >= t
+      // only when j >= t (j > t under the strict mask)
       const bool diag = p.causal && it.i == x.jb && it.qt == x.kt;
       if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
       // the loader's -lse and D for this stage are visible once its phase
@@ -813,8 +860,8 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
                   e0, e1);
         float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
         if (diag) {
-          p0 = (2 * j < t) ? 0.f : p0;
-          p1 = (2 * j + 1 < t) ? 0.f : p1;
+          p0 = (2 * j < t + p.diag_shift) ? 0.f : p0;
+          p1 = (2 * j + 1 < t + p.diag_shift) ? 0.f : p1;
         }
         pk[j] = pack_bf16x2(p0, p1);
       }
@@ -849,8 +896,13 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
     const long long off =
         ((static_cast<long long>(x.b) * p.L + static_cast<long long>(x.jb) * p.blk_len + krow) * p.Hkv +
          x.kvh) * D;
-    store_acc_row<D>(t_dv, 1.f, p.dv + off, valid);
-    store_acc_row<D>(t_dk, p.scale, p.dk + off, valid);
+    if (p.dk_acc != nullptr) {
+      fold_acc_row<D>(t_dv, 1.f, p.dv_acc + off, p.fold_kv, nullptr, valid);
+      fold_acc_row<D>(t_dk, p.scale, p.dk_acc + off, p.fold_kv, nullptr, valid);
+    } else {
+      store_acc_row<D>(t_dv, 1.f, p.dv + off, valid);
+      store_acc_row<D>(t_dk, p.scale, p.dk + off, valid);
+    }
     tc_fence_before();
     mbar_arrive(br.acc_free());
     ++units;
@@ -939,11 +991,16 @@ static cudaError_t launch_bwd_d(const BwdParams& prm, int num_sms, int max_ctas,
     if (max_ctas > 0 && max_ctas < g) g = max_ctas;
     return units < g ? units : g;
   };
-  ra_bwd_dq_kernel<D><<<grid_for(prm.units_dq), NUM_THREADS, QCfg<D>::SMEM_BYTES, stream>>>(prm);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  ra_bwd_dkdv_kernel<D><<<grid_for(prm.units_kv), NUM_THREADS, KCfg<D>::SMEM_BYTES, stream>>>(prm);
-  return cudaGetLastError();
+  if (prm.parts & 1) {
+    ra_bwd_dq_kernel<D><<<grid_for(prm.units_dq), NUM_THREADS, QCfg<D>::SMEM_BYTES, stream>>>(prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (prm.parts & 2) {
+    ra_bwd_dkdv_kernel<D><<<grid_for(prm.units_kv), NUM_THREADS, KCfg<D>::SMEM_BYTES, stream>>>(prm);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace bwd

@@ -64,6 +64,19 @@ struct BwdParams {
   float scale_log2;
   unsigned long long wait_limit_ns;
   unsigned debug_flags;
+  // Which kernels run: bit 0 the dQ kernel (also writes D), bit 1 the dK/dV
+  // kernel (reads D).  ring_attn_bwd runs both.
+  int parts;
+  // Per-visit launches (ring_attn_bwd_visit): when dq_acc / dk_acc are set,
+  // the dQ (dK, dV) rows are written to, or with fold_q (fold_kv) added to,
+  // these fp32 accumulators [B, L, H, d]; dq, if set, then receives the bf16
+  // rounding of the new dq_acc.  diag_shift = 1 makes the diagonal block
+  // exclude the key at the query's own row.
+  float* dq_acc;
+  float* dk_acc;
+  float* dv_acc;
+  int fold_q, fold_kv;
+  int diag_shift;
 };
 
 cudaError_t launch_fwd(const FwdParams& prm, int d, int grid, cudaStream_t stream);
@@ -76,6 +89,9 @@ constexpr long long kNoAllocScratchRows = 1ll << 20;
 // Address of that scratch on the current device (looked up once per device).
 cudaError_t noalloc_scratch(void** ptr);
 cudaError_t read_and_clear_status(unsigned long long* out);
+
+cudaError_t launch_round_bf16(const float* src, __nv_bfloat16* dst, long long n, int num_sms,
+                              cudaStream_t stream);
 
 cudaError_t launch_merge(const float* o_a, const float* lse_a, const float* o_b,
                          const float* lse_b, float* o_out, float* lse_out, long long rows, int d,

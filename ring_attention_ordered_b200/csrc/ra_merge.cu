@@ -76,6 +76,33 @@ __global__ void __launch_bounds__(MERGE_THREADS) ra_merge_kernel(
   }
 }
 
+// fp32 -> bf16, round to nearest even: 8 elements (32 bytes in, 16 out) per
+// thread and loop trip, grid-stride.
+__global__ void __launch_bounds__(256) ra_round_bf16_kernel(const float4* __restrict__ src,
+                                                            uint4* __restrict__ dst, long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * 256) {
+    const float4 a = src[2 * i], b = src[2 * i + 1];
+    uint4 o;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o.x) : "f"(a.y), "f"(a.x));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o.y) : "f"(a.w), "f"(a.z));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o.z) : "f"(b.y), "f"(b.x));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o.w) : "f"(b.w), "f"(b.z));
+    dst[i] = o;
+  }
+}
+
+cudaError_t launch_round_bf16(const float* src, __nv_bfloat16* dst, long long n, int num_sms,
+                              cudaStream_t stream) {
+  const long long n8 = n / 8;
+  long long grid = (n8 + 255) / 256;
+  if (grid > static_cast<long long>(num_sms) * 8) grid = static_cast<long long>(num_sms) * 8;
+  if (grid < 1) grid = 1;
+  ra_round_bf16_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(src), reinterpret_cast<uint4*>(dst), n8);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_merge(const float* o_a, const float* lse_a, const float* o_b,
                          const float* lse_b, float* o_out, float* lse_out, long long rows, int d,
                          int num_sms, cudaStream_t stream) {

@@ -34,6 +34,12 @@ into the fp32 accumulator in its epilogue.  The exchange uses
 torch.distributed point-to-point ops (NCCL between GPUs, gloo between CPU
 processes).  There is no other compute path: without the CUDA library the
 default visit raises.
+
+The backward pass (``ring_attention_bwd``) walks the same plan: each step a
+host adds its query block's dQ share (``ring_attn_bwd_visit``, dQ half) and
+then its share of the held block's dK, dV to fp32 accumulators that travel
+with the K/V block; one extra hop after the last step brings every block's
+accumulators home, where ``ring_attn_round_bf16`` rounds them.
 """
 
 from __future__ import annotations
@@ -274,3 +280,152 @@ def ring_attention_emulated(q, k, v, world: int, causal: bool, scale: float | No
         outs.append(o)
         lses.append(l)
     return unshard(outs, layout), unshard_lse(lses, layout)
+
+
+# ------------------------------------------------------------------ backward
+
+def cuda_bwd_visit(q, k, v, out, dout, lse, ws, mask, parts, dq_acc, dk_acc, dv_acc, scale, dq):
+    """One backward chunk-pair visit through the C ABI (ring_attn_bwd_visit);
+    the accumulators start at zero and every visit adds its share."""
+    from . import api
+    api.bwd_visit(q, k, v, out, dout, lse, ws, mask, parts, dq_acc, dk_acc, dv_acc, True, True,
+                  scale, dq)
+
+
+def cuda_round(src, like):
+    """A travelling fp32 gradient accumulator, home, rounded to bf16 (C ABI)."""
+    from . import api
+    return api.round_bf16(src)
+
+
+def _last_visits(plan):
+    last = {}
+    for t, (_, visits) in enumerate(plan):
+        for n, vi in enumerate(visits):
+            last[vi.qc] = (t, n)
+    return last
+
+
+def _bwd_phase(part, t, visits, last_q, q, out, dout, lse, ws, kb, vb, dq_acc, dq, dk_acc, dv_acc,
+               scale, visit):
+    for n, vi in enumerate(visits):
+        if part == 1:
+            visit(q[vi.qc], kb[vi.kc], vb[vi.kc], out[vi.qc], dout[vi.qc], lse[vi.qc], ws[vi.qc],
+                  vi.mask, 1, dq_acc[vi.qc], None, None, scale,
+                  dq[vi.qc] if last_q[vi.qc] == (t, n) else None)
+        else:
+            visit(q[vi.qc], kb[vi.kc], vb[vi.kc], out[vi.qc], dout[vi.qc], lse[vi.qc], ws[vi.qc],
+                  vi.mask, 2, None, dk_acc[vi.kc], dv_acc[vi.kc], scale, None)
+
+
+def _workspaces(q):
+    C, B, c, Hq, _ = q.shape
+    return [torch.empty(max(16, B * Hq * c * 4), dtype=torch.uint8, device=q.device)
+            for _ in range(C)]
+
+
+def ring_attention_bwd(q, k, v, out, dout, lse, causal: bool, scale: float | None = None,
+                       layout: str = "contiguous", group=None, visit=None, finish=None):
+    """This process's share of the ring attention backward pass over a
+    torch.distributed group.
+
+    q, out, dout [C, B, c, Hq, d], k, v [C, B, c, Hkv, d] and lse
+    [C, B, Hq, c] are this host's rows (``shard``; ``out`` and ``lse`` as
+    ``ring_attention`` returned them, 4-d / 3-d for C = 1).  Every ring step
+    the host computes its query block's dQ share against the K/V block it
+    holds, then adds its dK, dV share to that block's fp32 accumulators, which
+    travel around the ring with K and V (received from host i-1, passed to
+    host i+1); after the last step one more hop brings each block's
+    accumulators home, where they are rounded to bf16.  The K/V transfer of
+    step t+1 overlaps step t; the accumulators of a step are received while
+    the dQ half of the step computes.  Returns (dq, dk, dv) in the layout of
+    q, k, v.  ``visit``/``finish`` replace the CUDA visit and rounding
+    (tests on CPU processes)."""
+    squeeze = q.dim() == 4
+    if squeeze:
+        q, k, v, out, dout = (x.unsqueeze(0) for x in (q, k, v, out, dout))
+        lse = lse.unsqueeze(0)
+    visit = visit or cuda_bwd_visit
+    finish = finish or cuda_round
+    ring = P2PRing(group)
+    N = ring.world
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    plan = visit_plan(ring.rank, N, causal, layout)
+    last_q = _last_visits(plan)
+    dq_acc = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
+    dq = torch.empty_like(q)
+    ws = _workspaces(q)
+    acc = [(torch.zeros(k.shape, dtype=torch.float32, device=k.device),
+            torch.zeros(v.shape, dtype=torch.float32, device=v.device)),
+           (torch.empty(k.shape, dtype=torch.float32, device=k.device),
+            torch.empty(v.shape, dtype=torch.float32, device=v.device))]
+    held = [(k, v)]
+    spare = []
+    acc_wait = None
+    for t, (_, visits) in enumerate(plan):
+        kv_wait = None
+        if t < N - 1:
+            if len(spare) < 2:
+                spare.append((torch.empty_like(k), torch.empty_like(v)))
+            nk, nv = spare[t % 2]
+            kv_wait = ring.start(list(held[t]), [nk, nv])
+            held.append((nk, nv))
+        kb, vb = held[t]
+        dka, dva = acc[t % 2]
+        _bwd_phase(1, t, visits, last_q, q, out, dout, lse, ws, kb, vb, dq_acc, dq, dka, dva,
+                   scale, visit)
+        if acc_wait is not None:
+            acc_wait()          # this block's accumulators, from host i-1
+        _bwd_phase(2, t, visits, last_q, q, out, dout, lse, ws, kb, vb, dq_acc, dq, dka, dva,
+                   scale, visit)
+        if N > 1:
+            acc_wait = ring.start([dka, dva], list(acc[(t + 1) % 2]))
+        if kv_wait is not None:
+            kv_wait()
+    if acc_wait is not None:
+        acc_wait()              # this host's own block, home after N hops
+    fk, fv = acc[N % 2] if N > 1 else acc[0]
+    dk, dv = finish(fk, k), finish(fv, v)
+    if squeeze:
+        return dq[0], dk[0], dv[0]
+    return dq, dk, dv
+
+
+def ring_attention_bwd_emulated(q, k, v, out, dout, lse, world: int, causal: bool,
+                                scale: float | None = None, layout: str = "contiguous",
+                                visit=None, finish=None):
+    """All hosts of ``ring_attention_bwd`` on one device, whole-sequence
+    tensors in (q, out, dout [B, L, Hq, d], k, v [B, L, Hkv, d], lse
+    [B, Hq, L]) and out: every host runs exactly its visits, each K/V block's
+    accumulators receive the hosts' shares in the ring's order (host j at
+    step 0, j+1 at step 1, ...), without the exchange."""
+    visit = visit or cuda_bwd_visit
+    finish = finish or cuda_round
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    sh = lambda x, h: shard(x, h, world, layout)  # noqa: E731
+    lse_rows = lse.permute(0, 2, 1).unsqueeze(-1)          # [B, L, Hq, 1]
+    hosts = []
+    for h in range(world):
+        qh = sh(q, h)
+        hosts.append(dict(
+            q=qh, out=sh(out, h), dout=sh(dout, h),
+            lse=sh(lse_rows, h)[..., 0].permute(0, 1, 3, 2).contiguous(),
+            k=sh(k, h), v=sh(v, h), ws=_workspaces(qh),
+            dq_acc=torch.zeros(qh.shape, dtype=torch.float32, device=q.device),
+            dq=torch.empty_like(qh), plan=visit_plan(h, world, causal, layout)))
+    for hd in hosts:
+        hd["last_q"] = _last_visits(hd["plan"])
+    acc = [(torch.zeros(hd["k"].shape, dtype=torch.float32, device=k.device),
+            torch.zeros(hd["v"].shape, dtype=torch.float32, device=v.device)) for hd in hosts]
+    for t in range(world):
+        for part in (1, 2):
+            for hd in hosts:
+                j, visits = hd["plan"][t]
+                kb, vb = hosts[j]["k"], hosts[j]["v"]
+                _bwd_phase(part, t, visits, hd["last_q"], hd["q"], hd["out"], hd["dout"],
+                           hd["lse"], hd["ws"], kb, vb, hd["dq_acc"], hd["dq"], acc[j][0],
+                           acc[j][1], scale, visit)
+    dq = unshard([hd["dq"] for hd in hosts], layout)
+    dk = unshard([finish(acc[h][0], hosts[h]["k"]) for h in range(world)], layout)
+    dv = unshard([finish(acc[h][1], hosts[h]["v"]) for h in range(world)], layout)
+    return dq, dk, dv

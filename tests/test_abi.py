@@ -46,7 +46,7 @@ def test_status_strings_and_version(lib):
                                  "RA_ERR_CUDA", "RA_ERR_TIMEOUT"]):
         assert _lib.status_string(code) == name
     assert _lib.status_string(99) == "RA_ERR_UNKNOWN"
-    assert _lib.ring_attn_version() == 102
+    assert _lib.ring_attn_version() == 103
 
 
 # Fake, never-dereferenced device addresses: validation rejects these calls
@@ -218,3 +218,41 @@ def test_bwd_rejects_invalid_arguments(lib, kw, status):
 def test_bwd_empty_problem_launches_nothing(lib, kw):
     assert bwd_status(lib, q=0, k=0, v=0, out=0, dout=0, lse=0, dq=0, dk=0, dv=0, ws=0,
                       ws_bytes=0, **kw) == _lib.RA_OK
+
+
+def bwd_visit_status(lib, **kw):
+    args = dict(q=Q, k=K, v=V, out=O, dout=DO, lse=LSE, dq_acc=DQ, dk_acc=DK, dv_acc=DV, dq=0,
+                ws=WS, ws_bytes=1 << 20, B=1, Hq=2, Hkv=2, l=512, d=128, diag=1, parts=3,
+                fold_q=1, fold_kv=1, scale=0.088)
+    args.update(kw)
+    a = args
+    return lib.ring_attn_bwd_visit(a["q"], a["k"], a["v"], a["out"], a["dout"], a["lse"],
+                                   a["dq_acc"], a["dk_acc"], a["dv_acc"], a["dq"], a["ws"],
+                                   a["ws_bytes"], a["B"], a["Hq"], a["Hkv"], a["l"], a["d"],
+                                   a["diag"], a["parts"], a["fold_q"], a["fold_kv"], a["scale"],
+                                   None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(diag=3), _lib.RA_ERR_INVALID_ARG),
+    (dict(parts=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(parts=4), _lib.RA_ERR_INVALID_ARG),
+    (dict(fold_q=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(d=96), _lib.RA_ERR_UNSUPPORTED),
+    (dict(parts=1, dq_acc=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(parts=2, dk_acc=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(ws_bytes=100), _lib.RA_ERR_INVALID_ARG),
+    (dict(dq_acc=DQ + 4), _lib.RA_ERR_INVALID_ARG),
+    (dict(dk_acc=K + 64), _lib.RA_ERR_INVALID_ARG),      # accumulator overlaps k
+    (dict(dv_acc=DK + 64), _lib.RA_ERR_INVALID_ARG),     # accumulators overlap
+])
+def test_bwd_visit_rejects_invalid_arguments(lib, kw, status):
+    assert bwd_visit_status(lib, **kw) == status
+    assert _lib.last_error()
+
+
+def test_round_bf16_validation(lib):
+    assert lib.ring_attn_round_bf16(DQ, DK, 0, None) == _lib.RA_OK
+    assert lib.ring_attn_round_bf16(DQ, DK, 12, None) == _lib.RA_ERR_INVALID_ARG      # n % 8
+    assert lib.ring_attn_round_bf16(DQ + 4, DK, 16, None) == _lib.RA_ERR_INVALID_ARG  # alignment
+    assert lib.ring_attn_round_bf16(DQ, DQ + 16, 16, None) == _lib.RA_ERR_INVALID_ARG  # overlap

@@ -152,3 +152,93 @@ def test_emulated_zigzag_ring_on_the_l8k_workload(ra):
     o_ref, l_ref = oracle.attention_rows(q, k, v, w.causal, w.scale, bhr)
     b, h, r = (torch.from_numpy(bhr[:, i]).cuda() for i in range(3))
     compare(out[b, r, h, :], lse[b, h, r], o_ref, l_ref, "l8k zigzag")
+
+
+# ------------------------------------------------------------------ backward
+
+def fwd_stats_bf16(q, k, v, causal, scale):
+    """Forward output (rounded to bf16) and lse of the oracle, as the inputs a
+    backward visit takes."""
+    o, l_ = oracle.attention(q, k, v, causal, scale)
+    return torch.from_numpy(o).to(torch.bfloat16), torch.from_numpy(l_).float()
+
+
+@pytest.mark.parametrize("mask", [0, 1, 2])
+@pytest.mark.parametrize("B,Hq,Hkv,l,d", [(1, 2, 2, 256, 128), (2, 4, 2, 200, 64),
+                                          (1, 3, 1, 384, 128)])
+def test_bwd_visit_matches_oracle(ra, B, Hq, Hkv, l, d, mask):
+    """Both halves of one backward visit against block_attention_bwd, on the
+    oracle's own forward output and lse; the accumulators start from values
+    already there (fold) and dq is the rounding of the new dq_acc."""
+    from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
+    from parity import compare_grad
+    q, k, v = make_inputs(B, Hq, Hkv, l, d, seed=200 + l + mask)
+    _, k2, v2 = make_inputs(B, Hq, Hkv, l, d, seed=300 + l + mask)   # another K/V block
+    do = make_grad_output(B, l, Hq, d, seed=200 + l)
+    scale = 1.0 / d ** 0.5
+    out, lse = fwd_stats_bf16(q, k, v, True, scale)
+    g = torch.Generator().manual_seed(5)
+    dq0 = torch.randn(q.shape, generator=g)
+    dk0, dv0 = torch.randn(k.shape, generator=g), torch.randn(k.shape, generator=g)
+    dq_acc, dk_acc, dv_acc = dq0.cuda(), dk0.cuda(), dv0.cuda()
+    dq = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(B * Hq * l * 4, dtype=torch.uint8, device="cuda")
+    qd, kd, vd, od, dod, ld = (t.cuda() for t in (q, k2, v2, out, do, lse))
+    ra.bwd_visit(qd, kd, vd, od, dod, ld, ws, mask, 1, dq_acc=dq_acc, fold_q=True, scale=scale,
+                 dq=dq)
+    ra.bwd_visit(qd, kd, vd, od, dod, ld, ws, mask, 2, dk_acc=dk_acc, dv_acc=dv_acc, fold_kv=True,
+                 scale=scale)
+    ra.check_status()
+    pq, pk, pv = oracle.block_attention_bwd(q, k2, v2, out, do, lse, scale, KIND[mask])
+    what = f"{(B, Hq, Hkv, l, d, mask)}"
+    compare_grad(dq_acc.cpu() - dq0, pq, what + " dq")
+    compare_grad(dk_acc.cpu() - dk0, pk, what + " dk")
+    compare_grad(dv_acc.cpu() - dv0, pv, what + " dv")
+    assert torch.equal(dq, dq_acc.to(torch.bfloat16))
+    # without fold the accumulators are overwritten, whatever they held
+    dq_acc2 = torch.full_like(dq_acc, float("nan"))
+    ra.bwd_visit(qd, kd, vd, od, dod, ld, ws, mask, 3, dq_acc=dq_acc2,
+                 dk_acc=torch.full_like(dk_acc, float("nan")),
+                 dv_acc=torch.full_like(dv_acc, float("nan")), scale=scale)
+    ra.check_status()
+    compare_grad(dq_acc2.cpu(), pq, what + " dq (write)")
+
+
+def test_round_bf16_is_round_to_nearest_even(ra):
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(1 << 16, generator=g) * 10.0
+    x[:8] = torch.tensor([float("inf"), -float("inf"), 0.0, -0.0, 1e-40, 3.0e38, 1.00390625,
+                          1.01171875])
+    y = ra.round_bf16(x.cuda())
+    ra.check_status()
+    assert torch.equal(y.cpu().view(torch.int16), x.to(torch.bfloat16).view(torch.int16))
+
+
+# (layout, world, causal, B, Hq, Hkv, L, d)
+RING_BWD_CASES = [
+    ("contiguous", 4, True, 1, 4, 2, 1024, 128),
+    ("zigzag", 4, True, 1, 4, 2, 1024, 128),
+    ("striped", 4, True, 1, 4, 2, 1024, 128),
+    ("zigzag", 3, False, 2, 2, 1, 1200, 64),
+    ("contiguous", 1, True, 1, 2, 2, 384, 128),
+    ("striped", 2, False, 1, 2, 2, 512, 128),
+]
+
+
+@pytest.mark.parametrize("layout,world,causal,B,Hq,Hkv,L,d", RING_BWD_CASES)
+def test_emulated_ring_bwd_matches_oracle(ra, layout, world, causal, B, Hq, Hkv, L, d):
+    """Every host's backward visits with the travelling dK, dV accumulators,
+    on one device, against the definition's gradients."""
+    from parity import compare_grad
+    from ring_attention_ordered_b200 import ring
+    from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
+    q, k, v = make_inputs(B, Hq, Hkv, L, d, seed=L + 7 * world)
+    do = make_grad_output(B, L, Hq, d, seed=L + 7 * world)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    out, lse = ring.ring_attention_emulated(qd, kd, vd, world, causal, layout=layout)
+    got = ring.ring_attention_bwd_emulated(qd, kd, vd, out, dod, lse, world, causal,
+                                           layout=layout)
+    ra.check_status()
+    want = oracle.attention_bwd(q, k, v, do, causal, 1.0 / d ** 0.5)
+    for g_, w_, n in zip(got, want, "qkv"):
+        compare_grad(g_, w_, f"{layout} N={world} causal={causal} d{n}")

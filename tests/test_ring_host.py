@@ -217,3 +217,78 @@ def test_a_dead_neighbour_ends_the_ring_with_an_error():
     codes, res = _spawn(_dying_rank, 2)
     assert codes[1] == 3
     assert res.get(0, "").startswith("raised"), res
+
+
+# ------------------------------------------------------------------ backward
+
+def oracle_bwd_visit(q, k, v, out, dout, lse, ws, mask, parts, dq_acc, dk_acc, dv_acc, scale, dq):
+    """The contract of ring_attn_bwd_visit (accumulators add the visit's
+    share), computed by the oracle's block_attention_bwd."""
+    pq, pk, pv = oracle.block_attention_bwd(q, k, v, out, dout, lse, scale, KIND[mask])
+    if parts & 1:
+        dq_acc += torch.from_numpy(pq).to(dq_acc.dtype)
+        if dq is not None:
+            dq.copy_(dq_acc.to(dq.dtype))
+    if parts & 2:
+        dk_acc += torch.from_numpy(pk).to(dk_acc.dtype)
+        dv_acc += torch.from_numpy(pv).to(dv_acc.dtype)
+
+
+def plain_finish(src, like):
+    return src.to(like.dtype)
+
+
+def bwd_inputs(B, L, Hq=4, Hkv=2, d=8, seed=8, causal=True, scale=0.3):
+    q, k, v = small_inputs(B=B, L=L, Hq=Hq, Hkv=Hkv, d=d, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    do = torch.randn((B, L, Hq, d), generator=g)
+    out, lse = oracle.attention(q, k, v, causal, scale)
+    return q, k, v, do, torch.from_numpy(out).float(), torch.from_numpy(lse).float()
+
+
+@pytest.mark.parametrize("layout", ring.LAYOUTS)
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulated_ring_bwd_with_oracle_visits_is_the_gradient(layout, world, causal):
+    q, k, v, do, out, lse = bwd_inputs(1, 24, causal=causal)
+    got = ring.ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal, 0.3, layout,
+                                           visit=oracle_bwd_visit, finish=plain_finish)
+    want = oracle.attention_bwd(q, k, v, do, causal, 0.3)
+    for g_, w_ in zip(got, want):
+        np.testing.assert_allclose(g_.numpy(), w_, rtol=0, atol=2e-5)
+
+
+def _ring_bwd_rank(rank, world, port, layout, causal, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        L = 8 * world * ring.n_chunks(layout)
+        q, k, v, do, out, lse = bwd_inputs(2, L, causal=causal)
+        sh = lambda x: ring.shard(x, rank, world, layout)  # noqa: E731
+        lse_h = sh(lse.permute(0, 2, 1).unsqueeze(-1))[..., 0].permute(0, 1, 3, 2).contiguous()
+        ks, vs = sh(k), sh(v)
+        k0, v0 = ks.clone(), vs.clone()
+        grads = ring.ring_attention_bwd(sh(q), ks, vs, sh(out), sh(do), lse_h, causal, 0.3, layout,
+                                        visit=oracle_bwd_visit, finish=plain_finish)
+        assert torch.equal(ks, k0) and torch.equal(vs, v0)
+        results[rank] = grads
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,layout,causal", [
+    (2, "contiguous", True), (3, "contiguous", False), (4, "zigzag", True), (3, "striped", True),
+])
+def test_gloo_ring_bwd_is_the_gradient(world, layout, causal):
+    """dK and dV accumulators travel the ring with their K/V block between
+    gloo processes and come home after N hops."""
+    codes, res = _spawn(_ring_bwd_rank, world, layout, causal)
+    assert codes == [0] * world, codes
+    L = 8 * world * ring.n_chunks(layout)
+    q, k, v, do, out, lse = bwd_inputs(2, L, causal=causal)
+    want = oracle.attention_bwd(q, k, v, do, causal, 0.3)
+    for i in range(3):
+        got = ring.unshard([res[r][i] for r in range(world)], layout)
+        np.testing.assert_allclose(got.numpy(), want[i], rtol=0, atol=2e-5)
