@@ -595,7 +595,13 @@ def run_ring_emulated(args, w):
     lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
     fused_ms = timed(lambda: api.fwd(q, k, v, N, w.causal, w.scale, out=out, lse=lse,
                                      stream=stream))
-    del out, lse
+    if not args.no_bwd:
+        from ring_attention_ordered_b200.inputs import make_grad_output
+        do_full = make_grad_output(w.B, w.L, w.Hq, w.d, w.seed).to(dev)
+        out_full, lse_full = out, lse
+        lse_rows = lse_full.permute(0, 2, 1).unsqueeze(-1)
+        bwd_fused_ms = timed(lambda: api.bwd(q, k, v, out_full, do_full, lse_full, N, w.causal,
+                                             w.scale, stream=stream))
     for layout in ring.LAYOUTS:
         ks = [ring.shard(k, h, N, layout) for h in range(N)]
         vs = [ring.shard(v, h, N, layout) for h in range(N)]
@@ -610,13 +616,44 @@ def run_ring_emulated(args, w):
             del qh
         crit = max(host_ms)
         tflops = w.flops() / (crit / 1e3) / 1e12
+        # the backward of the same ring, host by host: dQ halves, then dK/dV
+        # halves into the held block's accumulators (fresh zeros per step)
+        bwd_ms = []
+        if not args.no_bwd:
+            for host in range(N):
+                qh = ring.shard(q, host, N, layout)
+                oh = ring.shard(out_full, host, N, layout)
+                dh = ring.shard(do_full, host, N, layout)
+                lh = ring.shard(lse_rows, host, N, layout)[..., 0].permute(0, 1, 3, 2).contiguous()
+                plan = ring.visit_plan(host, N, w.causal, layout)
+                last_q = ring._last_visits(plan)
+                ws = ring._workspaces(qh)
+                dq_acc = torch.zeros(qh.shape, dtype=torch.float32, device=dev)
+                dq_out = torch.empty_like(qh)
+                acc_k = torch.zeros(ks[0].shape, dtype=torch.float32, device=dev)
+                acc_v = torch.zeros(ks[0].shape, dtype=torch.float32, device=dev)
+
+                def host_bwd():
+                    for t, (j, visits) in enumerate(plan):
+                        for part in (1, 2):
+                            ring._bwd_phase(part, t, visits, last_q, qh, oh, dh, lh, ws, ks[j],
+                                            vs[j], dq_acc, dq_out, acc_k, acc_v, w.scale,
+                                            ring.cuda_bwd_visit)
+
+                bwd_ms.append(timed(host_bwd))
+                del qh, oh, dh, lh, ws, dq_acc, dq_out, acc_k, acc_v
         print(json.dumps({
             "kind": "ring_emulated", "workload": w.describe(), "layout": layout, "hosts": N,
             "host_ms": host_ms, "host_launches": host_launches, "critical_ms": crit,
             "sum_ms": sum(host_ms), "job_TFLOP/s_compute_only": tflops,
             "per_gpu_frac_of_burst": tflops / N / peaks["bf16_tflops"],
             "fused_1gpu_ms": fused_ms,
-            "frac_of_fused_over_N": fused_ms / (N * crit)}), flush=True)
+            "frac_of_fused_over_N": fused_ms / (N * crit),
+            "bwd_host_ms": bwd_ms,
+            "bwd_fused_1gpu_ms": None if args.no_bwd else bwd_fused_ms,
+            "bwd_critical_ms": max(bwd_ms) if bwd_ms else None,
+            "bwd_job_TFLOP/s_compute_only": (2.5 * w.flops() / (max(bwd_ms) / 1e3) / 1e12
+                                             if bwd_ms else None)}), flush=True)
         del ks, vs
         torch.cuda.empty_cache()
     return 0
