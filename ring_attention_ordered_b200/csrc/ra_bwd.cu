@@ -38,6 +38,7 @@
 #include <mutex>
 
 #include "ptx_sm100.cuh"
+#include "ra_exp2.cuh"
 #include "ra_internal.h"
 #include "ra_sync.cuh"
 #include "ring_attn.h"
@@ -48,10 +49,24 @@ namespace bwd {
 constexpr int TM = 128;              // rows per tile (queries or keys)
 constexpr int BOX_COLS = 64;
 constexpr int BOX_BYTES = 128 * 128;
-constexpr int NUM_THREADS = 192;     // softmax warpgroup, loader warp, MMA warp
-constexpr int WARP_LOAD = 4;
-constexpr int WARP_MMA = 5;
+// Two softmax warpgroups split each tile's 128 columns (64 each; both cover
+// all 128 TMEM lanes, so every SM sub-partition runs two of their warps and
+// one hides the other's TMEM and MUFU latency), then the loader and MMA warps.
+constexpr int NUM_THREADS = 320;
+constexpr int SOFTMAX_THREADS = 256;
+constexpr int WARP_LOAD = 8;
+constexpr int WARP_MMA = 9;
+constexpr int HALF = 64;             // columns per softmax warpgroup
 constexpr float LOG2E = 1.4426950408889634f;
+// Column pairs j (of a warpgroup's 32) with j % EMU == EMU - 1 take 2^x from
+// the polynomial on the FMA pipe, the others from MUFU ex2 (0, the default:
+// all from MUFU; one pair in 4, 3 or 2 on the polynomial measured 1-4%
+// slower on B200).
+#ifndef RA_BWD_EMU_PERIOD
+#define RA_BWD_EMU_PERIOD 0
+#endif
+constexpr int EMU = RA_BWD_EMU_PERIOD;
+
 
 // Device status word of the backward kernels: 0 = ok, else (code << 32) | where.
 __device__ unsigned long long g_status = 0ull;
@@ -90,17 +105,19 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d, uint32_t a, uint32_t b, u
 
 // Accumulating MMA with A (bf16 pairs, 128 along K) in TMEM and B MN-major in
 // shared memory (K = 128 rows of 128 bytes per 64-column box): 8 steps of
-// 16, A advancing 8 columns, B 16 rows (2048 bytes) per step.
-__device__ __forceinline__ void mma_tmem_a(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t hi,
-                                           uint32_t idesc, uint32_t acc) {
+// 16, B advancing 16 rows (2048 bytes) per step.  A was written by the two
+// softmax warpgroups into their own halves of a 128-column TMEM region: K
+// rows 0-63 as pairs at columns 0-31 of the region, rows 64-127 at 64-95.
+__device__ __forceinline__ void mma_tmem_a_split(uint32_t d, uint32_t a_tmem, uint32_t b,
+                                                 uint32_t hi, uint32_t idesc, uint32_t acc) {
   if (elect_one()) mma_ts<0, 0>(d, a_tmem, b, hi, idesc, acc);
   if (elect_one()) mma_ts<8, 128>(d, a_tmem, b, hi, idesc, 1u);
   if (elect_one()) mma_ts<16, 256>(d, a_tmem, b, hi, idesc, 1u);
   if (elect_one()) mma_ts<24, 384>(d, a_tmem, b, hi, idesc, 1u);
-  if (elect_one()) mma_ts<32, 512>(d, a_tmem, b, hi, idesc, 1u);
-  if (elect_one()) mma_ts<40, 640>(d, a_tmem, b, hi, idesc, 1u);
-  if (elect_one()) mma_ts<48, 768>(d, a_tmem, b, hi, idesc, 1u);
-  if (elect_one()) mma_ts<56, 896>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<64, 512>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<72, 640>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<80, 768>(d, a_tmem, b, hi, idesc, 1u);
+  if (elect_one()) mma_ts<88, 896>(d, a_tmem, b, hi, idesc, 1u);
 }
 
 __device__ __forceinline__ void commit(uint32_t bar) {
@@ -199,14 +216,19 @@ __device__ __forceinline__ void ds_chunk(const uint32_t (&pk)[16], const uint32_
 template <int D>
 struct QCfg {
   static constexpr int TILE = TM * D * 2;
-  static constexpr int NS = (D == 128) ? 2 : 4;       // K/V stages (K and V tile each)
+  // K tiles are read by S (early in a step) and by dQ (late), V tiles only by
+  // dP: three K stages let the next-but-one K tile load while dQ still reads
+  // the current one, two V stages suffice
+  static constexpr int NK = (D == 128) ? 3 : 6;
+  static constexpr int NV = (D == 128) ? 2 : 4;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = TILE;
-  static constexpr int OFF_KV = 2 * TILE;
-  static constexpr int OFF_BAR = OFF_KV + NS * 2 * TILE;
-  // qo_full, qo_empty, kv_full[NS], kv_empty[NS], s_full, s_free, dp_full,
-  // ds_full, acc_done, acc_free, drain
-  static constexpr int NUM_BARS = 2 + 2 * NS + 7;
+  static constexpr int OFF_K = 2 * TILE;
+  static constexpr int OFF_V = OFF_K + NK * TILE;
+  static constexpr int OFF_BAR = OFF_V + NV * TILE;
+  // qo_full, qo_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
+  // s_full, s_free, dp_full, ds_full, acc_done, acc_free, drain
+  static constexpr int NUM_BARS = 2 + 2 * NK + 2 * NV + 7;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -214,12 +236,16 @@ struct QCfg {
 
 struct QBars {
   uint32_t base;
-  int ns;
+  int nk, nv;
   __device__ __forceinline__ uint32_t qo_full() const { return base; }
   __device__ __forceinline__ uint32_t qo_empty() const { return base + 8; }
-  __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 16 + 8u * s; }
-  __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 16 + 8u * (ns + s); }
-  __device__ __forceinline__ uint32_t s_full() const { return base + 16 + 16u * ns; }
+  __device__ __forceinline__ uint32_t k_full(int s) const { return base + 16 + 8u * s; }
+  __device__ __forceinline__ uint32_t k_empty(int s) const { return base + 16 + 8u * (nk + s); }
+  __device__ __forceinline__ uint32_t v_full(int s) const { return base + 16 + 16u * nk + 8u * s; }
+  __device__ __forceinline__ uint32_t v_empty(int s) const {
+    return base + 16 + 16u * nk + 8u * (nv + s);
+  }
+  __device__ __forceinline__ uint32_t s_full() const { return base + 16 + 16u * nk + 16u * nv; }
   __device__ __forceinline__ uint32_t s_free() const { return s_full() + 8; }
   __device__ __forceinline__ uint32_t dp_full() const { return s_full() + 16; }
   __device__ __forceinline__ uint32_t ds_full() const { return s_full() + 24; }
@@ -298,19 +324,24 @@ __device__ void dq_loader(const BwdParams& p, const QBars& br, uint32_t base, co
     it.start(p, x);
     const int kvh = x.h / p.group;
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
-      const int s = kv_it % C::NS;
-      const uint32_t ph = (kv_it / C::NS) & 1u;
-      if (!wait_warp(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
       const int row = x.b * p.L + it.jb * p.blk_len + it.kl * TM;
-      const uint32_t dst = base + C::OFF_KV + s * 2 * C::TILE;
+      const int sk = kv_it % C::NK, sv = kv_it % C::NV;
+      if (!wait_warp(br.k_empty(sk), ((kv_it / C::NK) & 1u) ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
       if (elect_one()) {
-        mbar_arrive_expect_tx(br.kv_full(s), 2 * C::TILE);
+        mbar_arrive_expect_tx(br.k_full(sk), C::TILE);
 #pragma unroll
-        for (int bx = 0; bx < NBOX; ++bx) {
-          tma_load_3d(dst + bx * BOX_BYTES, &p.tm_k, br.kv_full(s), bx * BOX_COLS, kvh, row);
-          tma_load_3d(dst + C::TILE + bx * BOX_BYTES, &p.tm_v, br.kv_full(s), bx * BOX_COLS, kvh,
-                      row);
-        }
+        for (int bx = 0; bx < NBOX; ++bx)
+          tma_load_3d(base + C::OFF_K + sk * C::TILE + bx * BOX_BYTES, &p.tm_k, br.k_full(sk),
+                      bx * BOX_COLS, kvh, row);
+      }
+      __syncwarp();
+      if (!wait_warp(br.v_empty(sv), ((kv_it / C::NV) & 1u) ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.v_full(sv), C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx)
+          tma_load_3d(base + C::OFF_V + sv * C::TILE + bx * BOX_BYTES, &p.tm_v, br.v_full(sv),
+                      bx * BOX_COLS, kvh, row);
       }
       __syncwarp();
       ++kv_it;
@@ -319,10 +350,16 @@ __device__ void dq_loader(const BwdParams& p, const QBars& br, uint32_t base, co
   return;
 drain:
   if ((threadIdx.x & 31) == 0) {
-    const uint32_t n = kv_it < static_cast<uint32_t>(C::NS) ? kv_it : C::NS;
-    for (uint32_t i = 0; i < n; ++i) {
+    // let the copies already issued land before the CTA's shared memory goes
+    const uint32_t nk = kv_it < static_cast<uint32_t>(C::NK) ? kv_it : C::NK;
+    for (uint32_t i = 0; i < nk; ++i) {
       const uint32_t it = kv_it - 1 - i;
-      drain_wait(br.kv_full(it % C::NS), (it / C::NS) & 1u, 200000000ull);
+      drain_wait(br.k_full(it % C::NK), (it / C::NK) & 1u, 200000000ull);
+    }
+    const uint32_t nv = kv_it < static_cast<uint32_t>(C::NV) ? kv_it : C::NV;
+    for (uint32_t i = 0; i < nv; ++i) {
+      const uint32_t it = kv_it - 1 - i;
+      drain_wait(br.v_full(it % C::NV), (it / C::NV) & 1u, 200000000ull);
     }
     if (qo_pending) drain_wait(br.qo_full(), (units - 1) & 1u, 200000000ull);
   }
@@ -338,18 +375,19 @@ __device__ void dq_mma(const BwdParams& p, const QBars& br, uint32_t base, uint3
   const int G = gridDim.x, c = blockIdx.x;
   const uint64_t dq0 = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
   const uint64_t ddo0 = smem_desc_sw128(base + C::OFF_DO, 16, 1024);
-  const uint64_t dk0 = smem_desc_sw128(base + C::OFF_KV, 16, 1024);
-  const uint64_t dkmn0 = smem_desc_sw128(base + C::OFF_KV, BOX_BYTES, 1024);
+  const uint64_t dk0 = smem_desc_sw128(base + C::OFF_K, 16, 1024);
+  const uint64_t dv0 = smem_desc_sw128(base + C::OFF_V, 16, 1024);
+  const uint64_t dkmn0 = smem_desc_sw128(base + C::OFF_K, BOX_BYTES, 1024);
   const uint32_t q_lo = static_cast<uint32_t>(dq0), do_lo = static_cast<uint32_t>(ddo0);
-  const uint32_t k_lo = static_cast<uint32_t>(dk0), kmn_lo = static_cast<uint32_t>(dkmn0);
+  const uint32_t k_lo = static_cast<uint32_t>(dk0), v_lo = static_cast<uint32_t>(dv0);
+  const uint32_t kmn_lo = static_cast<uint32_t>(dkmn0);
   const uint32_t hi = static_cast<uint32_t>(dk0 >> 32), mn_hi = static_cast<uint32_t>(dkmn0 >> 32);
   const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
   uint32_t kv_it = 0, units = 0, step = 0;
-  auto issue_s = [&](int s) {
-    mma_kmajor<D>(t_s, q_lo, k_lo + ((s * 2 * C::TILE) >> 4), hi, IDESC_S);
-  };
-  auto issue_dp = [&](int s) {
-    mma_kmajor<D>(t_dp, do_lo, k_lo + ((s * 2 * C::TILE + C::TILE) >> 4), hi, IDESC_S);
+  // S = Q K^T from K stage sk, dP = dO V^T from V stage sv (all K-major)
+  auto issue_s = [&](int sk) { mma_kmajor<D>(t_s, q_lo, k_lo + ((sk * C::TILE) >> 4), hi, IDESC_S); };
+  auto issue_dp = [&](int sv) {
+    mma_kmajor<D>(t_dp, do_lo, v_lo + ((sv * C::TILE) >> 4), hi, IDESC_S);
   };
   for (int k = 0;; ++k) {
     const int u = unit_for_round(k, G, c);
@@ -358,24 +396,27 @@ __device__ void dq_mma(const BwdParams& p, const QBars& br, uint32_t base, uint3
     const int n = x.n;
     if (!wait_warp(br.qo_full(), units & 1u, cx, SITE_QD_FULL)) goto drain;
     {
-      const int s = kv_it % C::NS;
-      if (!wait_warp(br.kv_full(s), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+      const int sk = kv_it % C::NK, sv = kv_it % C::NV;
+      if (!wait_warp(br.k_full(sk), (kv_it / C::NK) & 1u, cx, SITE_KV_FULL)) goto drain;
       tc_fence_after();
-      issue_s(s);
+      issue_s(sk);
       commit(br.s_full());
-      issue_dp(s);
+      if (!wait_warp(br.v_full(sv), (kv_it / C::NV) & 1u, cx, SITE_KV_FULL)) goto drain;
+      tc_fence_after();
+      issue_dp(sv);
       commit(br.dp_full());
+      commit(br.v_empty(sv));
     }
     for (int idx = 0; idx < n; ++idx) {
       const bool more = idx + 1 < n;
-      const int s = kv_it % C::NS;
-      const int s1 = (kv_it + 1) % C::NS;
+      const int sk = kv_it % C::NK;
+      const int sk1 = (kv_it + 1) % C::NK, sv1 = (kv_it + 1) % C::NV;
       if (more) {
         // S for the next K/V tile as soon as the softmax has read this one
         if (!wait_warp(br.s_free(), step & 1u, cx, SITE_S_FREE)) goto drain;
-        if (!wait_warp(br.kv_full(s1), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
+        if (!wait_warp(br.k_full(sk1), ((kv_it + 1) / C::NK) & 1u, cx, SITE_KV_FULL)) goto drain;
         tc_fence_after();
-        issue_s(s1);
+        issue_s(sk1);
         commit(br.s_full());
       }
       if (!wait_warp(br.ds_full(), step & 1u, cx, SITE_DS_FULL)) goto drain;
@@ -383,11 +424,15 @@ __device__ void dq_mma(const BwdParams& p, const QBars& br, uint32_t base, uint3
           !wait_warp(br.acc_free(), (units - 1) & 1u, cx, SITE_ACC_FREE))
         goto drain;
       tc_fence_after();
-      mma_tmem_a(t_dq, t_dp, kmn_lo + ((s * 2 * C::TILE) >> 4), mn_hi, IDESC_DQ, idx > 0 ? 1u : 0u);
-      commit(br.kv_empty(s));
+      mma_tmem_a_split(t_dq, t_dp, kmn_lo + ((sk * C::TILE) >> 4), mn_hi, IDESC_DQ,
+                       idx > 0 ? 1u : 0u);
+      commit(br.k_empty(sk));
       if (more) {
-        issue_dp(s1);
+        if (!wait_warp(br.v_full(sv1), ((kv_it + 1) / C::NV) & 1u, cx, SITE_KV_FULL)) goto drain;
+        tc_fence_after();
+        issue_dp(sv1);
         commit(br.dp_full());
+        commit(br.v_empty(sv1));
       }
       ++step;
       ++kv_it;
@@ -404,11 +449,16 @@ drain:
 }
 
 template <int D>
-__device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, const Ctl& cx) {
-  const int t = threadIdx.x;                       // row inside the query tile
-  const int quarter = t >> 5;
+__device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, int wg,
+                           const Ctl& cx) {
+  constexpr int D2 = D / 2;                        // dQ columns of this warpgroup
+  const int t = threadIdx.x & 127;                 // row inside the query tile
+  const int quarter = (threadIdx.x >> 5) & 3;
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t t_s = tmem + lane_off, t_dp = t_s + 128, t_dq = t_s + 256;
+  // this warpgroup's keys: columns [64 wg, 64 wg + 64) of S and of dP
+  const uint32_t t_s = tmem + lane_off + HALF * wg, t_dp = tmem + lane_off + 128 + HALF * wg;
+  const uint32_t t_dq = tmem + lane_off + 256 + D2 * wg;
+  const int col0 = HALF * wg;
   const float c2 = p.scale_log2;
   const int G = gridDim.x, c = blockIdx.x;
   uint32_t units = 0, step = 0;
@@ -420,7 +470,8 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, c
     const bool valid = qrow < p.blk_len;
     const long long grow = static_cast<long long>(x.blk) * p.blk_len + qrow;
     const long long vidx = (static_cast<long long>(x.b) * p.Hq + x.h) * p.L + grow;
-    // D = rowsum(dO * O) of this row, and the row's lse in base 2
+    // D = rowsum(dO * O) of this row (both warpgroups form it; the first
+    // stores it), and the row's lse in base 2
     float dvec = 0.f, nlse2 = -INFINITY;
     if (valid) {
       const long long off = ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D;
@@ -440,7 +491,7 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, c
         acc = fmaf(bf16hi(a.w), bf16hi(g.w), acc);
       }
       dvec = acc;
-      p.dvec[vidx] = acc;
+      if (wg == 0) p.dvec[vidx] = acc;
       nlse2 = -p.lse[vidx] * LOG2E;
     }
     const uint64_t nl2 = f2_pack(nlse2, nlse2);
@@ -449,61 +500,72 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, c
     KvWalk it;
     it.start(p, x);
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
+      // keys allowed for this row: tile columns 0..lim
       int lim = min(TM, p.blk_len - it.kl * TM) - 1;
       if (p.causal && it.jb == x.blk) lim = min(lim, qrow - it.kl * TM - p.diag_shift);
-      const bool masked = __any_sync(0xffffffffu, lim < TM - 1);
+      const int lim_local = lim - col0;
+      const bool masked = __any_sync(0xffffffffu, lim_local < HALF - 1);
       if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
       tc_fence_after();
-      uint32_t sr[128];
+      uint32_t sr[64];
       tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(br.s_free());
       // P = 2^(s * scale * log2 e - lse * log2 e), rounded to bf16 pairs
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        float e0, e1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), c2x2,
-                         nl2),
-                  e0, e1);
-        float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+      for (int j = 0; j < 32; ++j) {
+        const uint64_t x2 =
+            f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), c2x2, nl2);
+        float p0, p1;
+        if (EMU > 0 && (j % (EMU > 0 ? EMU : 1)) == EMU - 1) {
+          exp2_poly2(x2, p0, p1);
+        } else {
+          float e0, e1;
+          f2_unpack(x2, e0, e1);
+          p0 = ex2_approx(e0);
+          p1 = ex2_approx(e1);
+        }
         if (masked) {
-          p0 = (2 * j > lim) ? 0.f : p0;
-          p1 = (2 * j + 1 > lim) ? 0.f : p1;
+          p0 = (2 * j > lim_local) ? 0.f : p0;
+          p1 = (2 * j + 1 > lim_local) ? 0.f : p1;
         }
         pk[j] = pack_bf16x2(p0, p1);
       }
       if (!wait_warp(br.dp_full(), step & 1u, cx, SITE_DP_FULL)) return;
       tc_fence_after();
-      // dS = P (dP - D) in four chunks of 32 keys, each stored as 16 columns
-      // of bf16 pairs over dP columns that have already been read
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t dp[32];
-        tmem_ld32(t_dp + 32 * cc, dp);
+      // dS = P (dP - D) in two chunks of 32 keys, each stored as 16 columns of
+      // bf16 pairs over this warpgroup's dP columns that have been read
+      {
+        // both 32-key chunks of dP are read before any dS pair overwrites them
+        uint32_t dp[2][32];
+        tmem_ld32(t_dp, dp[0]);
+        tmem_ld32(t_dp + 32, dp[1]);
         tmem_wait_ld();
-        uint32_t ds[16];
-        ds_chunk<false>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp, nullptr, dvec,
-                        ds);
-        tmem_st16(t_dp + 16 * cc, ds);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t ds[16];
+          ds_chunk<false>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp[cc], nullptr,
+                          dvec, ds);
+          tmem_st16(t_dp + 16 * cc, ds);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(br.ds_full());
       ++step;
     }
-    // epilogue: dQ = scale * (dS K) accumulated in TMEM
+    // epilogue: dQ = scale * (dS K) accumulated in TMEM, half the columns
     if (!wait_warp(br.acc_done(), units & 1u, cx, SITE_ACC_DONE)) return;
     tc_fence_after();
-    const long long qoff = ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D;
+    const long long qoff = ((static_cast<long long>(x.b) * p.L + grow) * p.Hq + x.h) * D + D2 * wg;
     if (p.dq_acc != nullptr)
-      fold_acc_row<D>(t_dq, p.scale, p.dq_acc + qoff, p.fold_q, p.dq ? p.dq + qoff : nullptr, valid);
+      fold_acc_row<D2>(t_dq, p.scale, p.dq_acc + qoff, p.fold_q, p.dq ? p.dq + qoff : nullptr,
+                       valid);
     else
-      store_acc_row<D>(t_dq, p.scale, p.dq + qoff, valid);
+      store_acc_row<D2>(t_dq, p.scale, p.dq + qoff, valid);
     tc_fence_before();
     mbar_arrive(br.acc_free());
     ++units;
@@ -519,21 +581,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_
   uint8_t* gen = smem_raw + (base - raw);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gen + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gen + C::OFF_MISC + 4);
-  const QBars br{base + C::OFF_BAR, C::NS};
+  const QBars br{base + C::OFF_BAR, C::NK, C::NV};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     mbar_init(br.qo_full(), 1);
     mbar_init(br.qo_empty(), 1);
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(br.kv_full(s), 1);
-      mbar_init(br.kv_empty(s), 1);
+    for (int s = 0; s < C::NK; ++s) {
+      mbar_init(br.k_full(s), 1);
+      mbar_init(br.k_empty(s), 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
+      mbar_init(br.v_full(s), 1);
+      mbar_init(br.v_empty(s), 1);
     }
     mbar_init(br.s_full(), 1);
-    mbar_init(br.s_free(), 128);
+    mbar_init(br.s_free(), SOFTMAX_THREADS);
     mbar_init(br.dp_full(), 1);
-    mbar_init(br.ds_full(), 128);
+    mbar_init(br.ds_full(), SOFTMAX_THREADS);
     mbar_init(br.acc_done(), 1);
-    mbar_init(br.acc_free(), 128);
+    mbar_init(br.acc_free(), SOFTMAX_THREADS);
     mbar_init(br.drain(), 1);
     *abort_flag = 0u;
     fence_mbarrier_init();
@@ -553,8 +619,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
-  if (warp < 4) {
-    dq_softmax<D>(p, br, tmem, cx);
+  if (warp < 8) {
+    dq_softmax<D>(p, br, tmem, warp >> 2, cx);
   } else if (warp == WARP_LOAD) {
     dq_loader<D>(p, br, base, cx);
   } else {
@@ -686,10 +752,26 @@ __device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, fl
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
       const int s = q_it % C::NS;
       const uint32_t ph = (q_it / C::NS) & 1u;
-      if (!wait_warp(br.qd_empty(s), ph ^ 1u, cx, SITE_QD_EMPTY)) goto drain;
       const int h = x.kvh * p.group + it.hh;
       const int row = x.b * p.L + it.i * p.blk_len + it.qt * TM;
       const uint32_t dst = base + C::OFF_ST + s * 2 * C::TILE;
+      // -lse * log2(e) and D of the tile's 128 query rows (rows past the
+      // block end: weight 0 through -inf, D = 0), loaded before the wait for
+      // the stage so that their latency overlaps it
+      const long long vbase = (static_cast<long long>(x.b) * p.Hq + h) * p.L +
+                              static_cast<long long>(it.i) * p.blk_len;
+      float nlr[TM / 32], dvr[TM / 32];
+#pragma unroll
+      for (int j = 0; j < TM / 32; ++j) {
+        const int qrow = it.qt * TM + lane + 32 * j;
+        nlr[j] = -INFINITY;
+        dvr[j] = 0.f;
+        if (qrow < p.blk_len) {
+          nlr[j] = -p.lse[vbase + qrow] * LOG2E;
+          dvr[j] = p.dvec[vbase + qrow];
+        }
+      }
+      if (!wait_warp(br.qd_empty(s), ph ^ 1u, cx, SITE_QD_EMPTY)) goto drain;
       if (elect_one()) {
         mbar_arrive_expect_tx(br.qd_full(s), 2 * C::TILE);
 #pragma unroll
@@ -698,22 +780,11 @@ __device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, fl
           tma_load_3d(dst + C::TILE + bx * BOX_BYTES, &p.tm_do, br.qd_full(s), bx * BOX_COLS, h, row);
         }
       }
-      // -lse * log2(e) and D of the tile's 128 query rows (rows past the
-      // block end: weight 0 through -inf, D = 0)
       float* vs = vec_smem + s * 2 * TM;
-      const long long vbase = (static_cast<long long>(x.b) * p.Hq + h) * p.L +
-                              static_cast<long long>(it.i) * p.blk_len;
 #pragma unroll
       for (int j = 0; j < TM / 32; ++j) {
-        const int r = lane + 32 * j;
-        const int qrow = it.qt * TM + r;
-        float nl = -INFINITY, dvv = 0.f;
-        if (qrow < p.blk_len) {
-          nl = -p.lse[vbase + qrow] * LOG2E;
-          dvv = p.dvec[vbase + qrow];
-        }
-        vs[r] = nl;
-        vs[TM + r] = dvv;
+        vs[lane + 32 * j] = nlr[j];
+        vs[TM + lane + 32 * j] = dvr[j];
       }
       mbar_arrive(br.qd_full(s));
       ++q_it;
@@ -780,7 +851,7 @@ __device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint3
         goto drain;
       tc_fence_after();
       // dV += P^T dO (dO MN-major)
-      mma_tmem_a(t_dv, t_s, stmn_lo + ((s * 2 * C::TILE + C::TILE) >> 4), mn_hi, IDESC_ACC,
+      mma_tmem_a_split(t_dv, t_s, stmn_lo + ((s * 2 * C::TILE + C::TILE) >> 4), mn_hi, IDESC_ACC,
                  idx > 0 ? 1u : 0u);
       if (more) {
         // S^T of the next step may overwrite P^T: the tensor pipe runs the
@@ -793,7 +864,7 @@ __device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint3
       if (!wait_warp(br.ds_full(), step & 1u, cx, SITE_DS_FULL)) goto drain;
       tc_fence_after();
       // dK += dS^T Q (Q MN-major)
-      mma_tmem_a(t_dk, t_dp, stmn_lo + ((s * 2 * C::TILE) >> 4), mn_hi, IDESC_ACC,
+      mma_tmem_a_split(t_dk, t_dp, stmn_lo + ((s * 2 * C::TILE) >> 4), mn_hi, IDESC_ACC,
                  idx > 0 ? 1u : 0u);
       commit(br.qd_empty(s));
       if (more) {
@@ -816,13 +887,16 @@ drain:
 
 template <int D>
 __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, const float* vec_smem,
-                           const Ctl& cx) {
+                           int wg, const Ctl& cx) {
   using C = KCfg<D>;
-  const int t = threadIdx.x;                       // key row inside the tile
-  const int quarter = t >> 5;
+  constexpr int D2 = D / 2;                        // dK, dV columns of this warpgroup
+  const int t = threadIdx.x & 127;                 // key row inside the tile
+  const int quarter = (threadIdx.x >> 5) & 3;
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t t_s = tmem + lane_off, t_dp = t_s + 128;
-  const uint32_t t_dv = t_s + 256, t_dk = t_s + 256 + D;
+  // this warpgroup's queries: columns [64 wg, 64 wg + 64) of S^T and dP^T
+  const uint32_t t_s = tmem + lane_off + HALF * wg, t_dp = tmem + lane_off + 128 + HALF * wg;
+  const uint32_t t_dv = tmem + lane_off + 256 + D2 * wg, t_dk = tmem + lane_off + 256 + D + D2 * wg;
+  const int col0 = HALF * wg;
   const uint64_t c2x2 = f2_pack(p.scale_log2, p.scale_log2);
   const int G = gridDim.x, c = blockIdx.x;
   uint32_t units = 0, step = 0, q_it = 0;
@@ -837,50 +911,60 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
       // the diagonal tile of the own block: query column j sees key row t
       // only when j >= t (j > t under the strict mask)
       const bool diag = p.causal && it.i == x.jb && it.qt == x.kt;
+      const int first = t + p.diag_shift - col0;   // first allowed local column
       if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
       // the loader's -lse and D for this stage are visible once its phase
       // completed (it completed before S^T was issued)
       if (!wait_warp(br.qd_full(s), (q_it / C::NS) & 1u, cx, SITE_QD_FULL)) return;
       tc_fence_after();
-      const float* nl = vec_smem + s * 2 * TM;
-      const float* dvv = nl + TM;
-      uint32_t sr[128];
+      const float* nl = vec_smem + s * 2 * TM + col0;
+      const float* dvv = vec_smem + s * 2 * TM + TM + col0;
+      uint32_t sr[64];
       tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
+      for (int j = 0; j < 32; ++j) {
         const float2 l2 = reinterpret_cast<const float2*>(nl)[j];
-        float e0, e1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), c2x2,
-                         f2_pack(l2.x, l2.y)),
-                  e0, e1);
-        float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])),
+                                   c2x2, f2_pack(l2.x, l2.y));
+        float p0, p1;
+        if (EMU > 0 && (j % (EMU > 0 ? EMU : 1)) == EMU - 1) {
+          exp2_poly2(x2, p0, p1);
+        } else {
+          float e0, e1;
+          f2_unpack(x2, e0, e1);
+          p0 = ex2_approx(e0);
+          p1 = ex2_approx(e1);
+        }
         if (diag) {
-          p0 = (2 * j < t + p.diag_shift) ? 0.f : p0;
-          p1 = (2 * j + 1 < t + p.diag_shift) ? 0.f : p1;
+          p0 = (2 * j < first) ? 0.f : p0;
+          p1 = (2 * j + 1 < first) ? 0.f : p1;
         }
         pk[j] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(t_s, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(t_s + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      // P^T as bf16 pairs over this warpgroup's own S^T columns
+      tmem_st32(t_s, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(br.p_full());
       if (!wait_warp(br.dp_full(), step & 1u, cx, SITE_DP_FULL)) return;
       tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t dp[32];
-        tmem_ld32(t_dp + 32 * cc, dp);
+      {
+        // both 32-query chunks of dP^T are read before any dS^T pair
+        // overwrites them
+        uint32_t dp[2][32];
+        tmem_ld32(t_dp, dp[0]);
+        tmem_ld32(t_dp + 32, dp[1]);
         tmem_wait_ld();
-        uint32_t ds[16];
-        ds_chunk<true>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp, dvv + 32 * cc,
-                       0.f, ds);
-        tmem_st16(t_dp + 16 * cc, ds);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t ds[16];
+          ds_chunk<true>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp[cc],
+                         dvv + 32 * cc, 0.f, ds);
+          tmem_st16(t_dp + 16 * cc, ds);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -888,20 +972,20 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
       ++step;
       ++q_it;
     }
-    // epilogue: dV and dK = scale * (dS^T Q) of this key tile
+    // epilogue: dV and dK = scale * (dS^T Q) of this key tile, half the columns
     if (!wait_warp(br.acc_done(), units & 1u, cx, SITE_ACC_DONE)) return;
     tc_fence_after();
     const int krow = x.kt * TM + t;
     const bool valid = krow < p.blk_len;
     const long long off =
         ((static_cast<long long>(x.b) * p.L + static_cast<long long>(x.jb) * p.blk_len + krow) * p.Hkv +
-         x.kvh) * D;
+         x.kvh) * D + D2 * wg;
     if (p.dk_acc != nullptr) {
-      fold_acc_row<D>(t_dv, 1.f, p.dv_acc + off, p.fold_kv, nullptr, valid);
-      fold_acc_row<D>(t_dk, p.scale, p.dk_acc + off, p.fold_kv, nullptr, valid);
+      fold_acc_row<D2>(t_dv, 1.f, p.dv_acc + off, p.fold_kv, nullptr, valid);
+      fold_acc_row<D2>(t_dk, p.scale, p.dk_acc + off, p.fold_kv, nullptr, valid);
     } else {
-      store_acc_row<D>(t_dv, 1.f, p.dv + off, valid);
-      store_acc_row<D>(t_dk, p.scale, p.dk + off, valid);
+      store_acc_row<D2>(t_dv, 1.f, p.dv + off, valid);
+      store_acc_row<D2>(t_dk, p.scale, p.dk + off, valid);
     }
     tc_fence_before();
     mbar_arrive(br.acc_free());
@@ -930,10 +1014,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __gri
     }
     mbar_init(br.s_full(), 1);
     mbar_init(br.dp_full(), 1);
-    mbar_init(br.p_full(), 128);
-    mbar_init(br.ds_full(), 128);
+    mbar_init(br.p_full(), SOFTMAX_THREADS);
+    mbar_init(br.ds_full(), SOFTMAX_THREADS);
     mbar_init(br.acc_done(), 1);
-    mbar_init(br.acc_free(), 128);
+    mbar_init(br.acc_free(), SOFTMAX_THREADS);
     mbar_init(br.drain(), 1);
     *abort_flag = 0u;
     fence_mbarrier_init();
@@ -953,8 +1037,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
-  if (warp < 4) {
-    kv_softmax<D>(p, br, tmem, vec_smem, cx);
+  if (warp < 8) {
+    kv_softmax<D>(p, br, tmem, vec_smem, warp >> 2, cx);
   } else if (warp == WARP_LOAD) {
     kv_loader<D>(p, br, base, vec_smem, cx);
   } else {
