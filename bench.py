@@ -112,7 +112,8 @@ KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd.cu",
                   "ring_attention_ordered_b200/csrc/ra_api.cu",
                   "ring_attention_ordered_b200/csrc/ra_internal.h",
                   "ring_attention_ordered_b200/csrc/ra_merge_math.cuh",
-                  "ring_attention_ordered_b200/csrc/ra_sync.cuh"]
+                  "ring_attention_ordered_b200/csrc/ra_sync.cuh",
+                  "ring_attention_ordered_b200/csrc/ra_exp2.cuh"]
 TRAFFIC_RECORD = "profiles/ra_fwd_l128k_h32_causal_dram.md"
 
 

@@ -148,3 +148,29 @@ def test_bwd_short_workspace_is_rejected(ra):
     with pytest.raises(_lib.RingAttnError) as ei:
         ra.bwd(q, q.clone(), q.clone(), q.clone(), q.clone(), lse, 2, True, workspace=ws)
     assert ei.value.status == _lib.RA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,n_sample", [("l128k_h32_causal", 256), ("l1m_gqa4_sink_causal", 256)])
+def test_bwd_large_workloads_dq_rows(ra, name, n_sample):
+    """The 128K and the 1M-token (attention-sink, GQA) workloads at full
+    size: sampled dQ rows and rows at every ring-block boundary of the first
+    and last head against the oracle (each dQ row needs only its own scores);
+    dK and dV, which need every query row of a group, are checked on the
+    smaller workloads."""
+    from ring_attention_ordered_b200.inputs import WORKLOADS, make_grad_output, sample_rows, workload_inputs
+    w = WORKLOADS[name]
+    q, k, v = workload_inputs(w)
+    do = make_grad_output(w.B, w.L, w.Hq, w.d, w.seed)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    out, lse = ra.fwd(qd, kd, vd, w.n_ring, w.causal, w.scale)
+    dq, dk, dv = ra.bwd(qd, kd, vd, out, dod, lse, w.n_ring, w.causal, w.scale)
+    ra.check_status()
+    assert torch.isfinite(dk).all() and torch.isfinite(dv).all()
+    del qd, kd, vd, dod, out, lse, dk, dv
+    lb = w.block_len
+    edges = sorted({r for i in range(w.n_ring + 1) for r in (i * lb - 1, i * lb) if 0 <= r < w.L})
+    bhr = np.concatenate([sample_rows(w, n_sample, seed=w.seed + 1),
+                          np.array([[0, h, r] for h in (0, w.Hq - 1) for r in edges], np.int64)])
+    ref = oracle.attention_bwd_dq_rows(q, k, v, do, w.causal, w.scale, bhr)
+    b, h, r = (torch.from_numpy(bhr[:, i]).cuda() for i in range(3))
+    compare_grad(dq[b, r, h, :], ref, f"{name} dQ rows")
