@@ -641,32 +641,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_
 template <int D>
 struct KCfg {
   static constexpr int TILE = TM * D * 2;
-  static constexpr int NS = (D == 128) ? 2 : 4;       // Q/dO stages
+  // Q tiles are read by S^T early in a step (the next tile's S^T overlaps the
+  // current exponentials) and by dK late, so Q needs three stages; dO is read
+  // by dP^T and dV within one step, two stages
+  static constexpr int NQ = (D == 128) ? 3 : 6;
+  static constexpr int NO = (D == 128) ? 2 : 4;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = TILE;
-  static constexpr int OFF_ST = 2 * TILE;             // stage s: Q, then dO
-  static constexpr int OFF_VEC = OFF_ST + NS * 2 * TILE;  // stage s: -lse*log2e [128], D [128]
-  static constexpr int VEC_BYTES = 2 * TM * 4;
-  static constexpr int OFF_BAR = OFF_VEC + NS * VEC_BYTES;
-  // kv_full, kv_empty, qd_full[NS], qd_empty[NS], s_full, dp_full, p_full,
-  // ds_full, acc_done, acc_free, drain
-  static constexpr int NUM_BARS = 2 + 2 * NS + 7;
+  static constexpr int OFF_Q = 2 * TILE;
+  static constexpr int OFF_DO = OFF_Q + NQ * TILE;
+  static constexpr int OFF_LSE = OFF_DO + NO * TILE;    // per Q stage: -lse*log2e [128]
+  static constexpr int OFF_DV = OFF_LSE + NQ * TM * 4;  // per dO stage: D [128]
+  static constexpr int OFF_BAR = OFF_DV + NO * TM * 4;
+  // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NO], do_empty[NO],
+  // s_full, dp_full, s_free, pd_full, acc_done, acc_free, drain
+  static constexpr int NUM_BARS = 2 + 2 * NQ + 2 * NO + 7;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // no alignment slack: the kernel checks that the dynamic shared memory
+  // starts on a 1024-byte boundary (the 128-byte swizzle needs it) and
+  // reports RA_ERR_UNSUPPORTED otherwise
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct KBars {
   uint32_t base;
-  int ns;
+  int nq, no;
   __device__ __forceinline__ uint32_t kv_full() const { return base; }
   __device__ __forceinline__ uint32_t kv_empty() const { return base + 8; }
-  __device__ __forceinline__ uint32_t qd_full(int s) const { return base + 16 + 8u * s; }
-  __device__ __forceinline__ uint32_t qd_empty(int s) const { return base + 16 + 8u * (ns + s); }
-  __device__ __forceinline__ uint32_t s_full() const { return base + 16 + 16u * ns; }
+  __device__ __forceinline__ uint32_t q_full(int s) const { return base + 16 + 8u * s; }
+  __device__ __forceinline__ uint32_t q_empty(int s) const { return base + 16 + 8u * (nq + s); }
+  __device__ __forceinline__ uint32_t do_full(int s) const { return base + 16 + 16u * nq + 8u * s; }
+  __device__ __forceinline__ uint32_t do_empty(int s) const {
+    return base + 16 + 16u * nq + 8u * (no + s);
+  }
+  __device__ __forceinline__ uint32_t s_full() const { return base + 16 + 16u * nq + 16u * no; }
   __device__ __forceinline__ uint32_t dp_full() const { return s_full() + 8; }
-  __device__ __forceinline__ uint32_t p_full() const { return s_full() + 16; }
-  __device__ __forceinline__ uint32_t ds_full() const { return s_full() + 24; }
+  __device__ __forceinline__ uint32_t s_free() const { return s_full() + 16; }
+  __device__ __forceinline__ uint32_t pd_full() const { return s_full() + 24; }
   __device__ __forceinline__ uint32_t acc_done() const { return s_full() + 32; }
   __device__ __forceinline__ uint32_t acc_free() const { return s_full() + 40; }
   __device__ __forceinline__ uint32_t drain() const { return s_full() + 48; }
@@ -720,8 +732,8 @@ struct QWalk {
 };
 
 template <int D>
-__device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, float* vec_smem,
-                          const Ctl& cx) {
+__device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, float* lse_smem,
+                          float* dv_smem, const Ctl& cx) {
   using C = KCfg<D>;
   constexpr int NBOX = D / BOX_COLS;
   const int lane = threadIdx.x & 31;
@@ -750,14 +762,12 @@ __device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, fl
     QWalk it;
     it.start(p, x);
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
-      const int s = q_it % C::NS;
-      const uint32_t ph = (q_it / C::NS) & 1u;
+      const int sq = q_it % C::NQ, so = q_it % C::NO;
       const int h = x.kvh * p.group + it.hh;
       const int row = x.b * p.L + it.i * p.blk_len + it.qt * TM;
-      const uint32_t dst = base + C::OFF_ST + s * 2 * C::TILE;
       // -lse * log2(e) and D of the tile's 128 query rows (rows past the
-      // block end: weight 0 through -inf, D = 0), loaded before the wait for
-      // the stage so that their latency overlaps it
+      // block end: weight 0 through -inf, D = 0), loaded before the waits
+      // for the stages so that their latency overlaps them
       const long long vbase = (static_cast<long long>(x.b) * p.Hq + h) * p.L +
                               static_cast<long long>(it.i) * p.blk_len;
       float nlr[TM / 32], dvr[TM / 32];
@@ -771,32 +781,44 @@ __device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, fl
           dvr[j] = p.dvec[vbase + qrow];
         }
       }
-      if (!wait_warp(br.qd_empty(s), ph ^ 1u, cx, SITE_QD_EMPTY)) goto drain;
+      if (!wait_warp(br.q_empty(sq), ((q_it / C::NQ) & 1u) ^ 1u, cx, SITE_QD_EMPTY)) goto drain;
       if (elect_one()) {
-        mbar_arrive_expect_tx(br.qd_full(s), 2 * C::TILE);
+        mbar_arrive_expect_tx(br.q_full(sq), C::TILE);
 #pragma unroll
-        for (int bx = 0; bx < NBOX; ++bx) {
-          tma_load_3d(dst + bx * BOX_BYTES, &p.tm_q, br.qd_full(s), bx * BOX_COLS, h, row);
-          tma_load_3d(dst + C::TILE + bx * BOX_BYTES, &p.tm_do, br.qd_full(s), bx * BOX_COLS, h, row);
-        }
+        for (int bx = 0; bx < NBOX; ++bx)
+          tma_load_3d(base + C::OFF_Q + sq * C::TILE + bx * BOX_BYTES, &p.tm_q, br.q_full(sq),
+                      bx * BOX_COLS, h, row);
       }
-      float* vs = vec_smem + s * 2 * TM;
 #pragma unroll
-      for (int j = 0; j < TM / 32; ++j) {
-        vs[lane + 32 * j] = nlr[j];
-        vs[TM + lane + 32 * j] = dvr[j];
+      for (int j = 0; j < TM / 32; ++j) lse_smem[sq * TM + lane + 32 * j] = nlr[j];
+      mbar_arrive(br.q_full(sq));
+      if (!wait_warp(br.do_empty(so), ((q_it / C::NO) & 1u) ^ 1u, cx, SITE_QD_EMPTY)) goto drain;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(br.do_full(so), C::TILE);
+#pragma unroll
+        for (int bx = 0; bx < NBOX; ++bx)
+          tma_load_3d(base + C::OFF_DO + so * C::TILE + bx * BOX_BYTES, &p.tm_do, br.do_full(so),
+                      bx * BOX_COLS, h, row);
       }
-      mbar_arrive(br.qd_full(s));
+#pragma unroll
+      for (int j = 0; j < TM / 32; ++j) dv_smem[so * TM + lane + 32 * j] = dvr[j];
+      mbar_arrive(br.do_full(so));
       ++q_it;
     }
   }
   return;
 drain:
   if (lane == 0) {
-    const uint32_t n = q_it < static_cast<uint32_t>(C::NS) ? q_it : C::NS;
-    for (uint32_t i = 0; i < n; ++i) {
+    // let the copies already issued land before the CTA's shared memory goes
+    const uint32_t nq = q_it < static_cast<uint32_t>(C::NQ) ? q_it : C::NQ;
+    for (uint32_t i = 0; i < nq; ++i) {
       const uint32_t it = q_it - 1 - i;
-      drain_wait(br.qd_full(it % C::NS), (it / C::NS) & 1u, 200000000ull);
+      drain_wait(br.q_full(it % C::NQ), (it / C::NQ) & 1u, 200000000ull);
+    }
+    const uint32_t no = q_it < static_cast<uint32_t>(C::NO) ? q_it : C::NO;
+    for (uint32_t i = 0; i < no; ++i) {
+      const uint32_t it = q_it - 1 - i;
+      drain_wait(br.do_full(it % C::NO), (it / C::NO) & 1u, 200000000ull);
     }
     if (kv_pending) drain_wait(br.kv_full(), (units - 1) & 1u, 200000000ull);
   }
@@ -812,19 +834,20 @@ __device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint3
   const int G = gridDim.x, c = blockIdx.x;
   const uint64_t dk0 = smem_desc_sw128(base + C::OFF_K, 16, 1024);
   const uint64_t dv0 = smem_desc_sw128(base + C::OFF_V, 16, 1024);
-  const uint64_t dst0 = smem_desc_sw128(base + C::OFF_ST, 16, 1024);
-  const uint64_t dstmn0 = smem_desc_sw128(base + C::OFF_ST, BOX_BYTES, 1024);
+  const uint64_t dq0 = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
+  const uint64_t ddo0 = smem_desc_sw128(base + C::OFF_DO, 16, 1024);
+  const uint64_t dqmn0 = smem_desc_sw128(base + C::OFF_Q, BOX_BYTES, 1024);
+  const uint64_t ddomn0 = smem_desc_sw128(base + C::OFF_DO, BOX_BYTES, 1024);
   const uint32_t k_lo = static_cast<uint32_t>(dk0), v_lo = static_cast<uint32_t>(dv0);
-  const uint32_t st_lo = static_cast<uint32_t>(dst0), stmn_lo = static_cast<uint32_t>(dstmn0);
-  const uint32_t hi = static_cast<uint32_t>(dk0 >> 32), mn_hi = static_cast<uint32_t>(dstmn0 >> 32);
+  const uint32_t q_lo = static_cast<uint32_t>(dq0), do_lo = static_cast<uint32_t>(ddo0);
+  const uint32_t qmn_lo = static_cast<uint32_t>(dqmn0), domn_lo = static_cast<uint32_t>(ddomn0);
+  const uint32_t hi = static_cast<uint32_t>(dk0 >> 32), mn_hi = static_cast<uint32_t>(dqmn0 >> 32);
   const uint32_t t_s = tmem, t_dp = tmem + 128, t_dv = tmem + 256, t_dk = tmem + 256 + D;
   uint32_t q_it = 0, units = 0, step = 0;
-  // S^T = K Q^T and dP^T = V dO^T for stage s (Q and dO K-major)
-  auto issue_s = [&](int s) {
-    mma_kmajor<D>(t_s, k_lo, st_lo + ((s * 2 * C::TILE) >> 4), hi, IDESC_S);
-  };
-  auto issue_dp = [&](int s) {
-    mma_kmajor<D>(t_dp, v_lo, st_lo + ((s * 2 * C::TILE + C::TILE) >> 4), hi, IDESC_S);
+  // S^T = K Q^T (Q stage sq) and dP^T = V dO^T (dO stage so), all K-major
+  auto issue_s = [&](int sq) { mma_kmajor<D>(t_s, k_lo, q_lo + ((sq * C::TILE) >> 4), hi, IDESC_S); };
+  auto issue_dp = [&](int so) {
+    mma_kmajor<D>(t_dp, v_lo, do_lo + ((so * C::TILE) >> 4), hi, IDESC_S);
   };
   for (int k = 0;; ++k) {
     const int u = unit_for_round(k, G, c);
@@ -833,42 +856,49 @@ __device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint3
     const int n = x.n;
     if (!wait_warp(br.kv_full(), units & 1u, cx, SITE_KV_FULL)) goto drain;
     {
-      const int s = q_it % C::NS;
-      if (!wait_warp(br.qd_full(s), (q_it / C::NS) & 1u, cx, SITE_QD_FULL)) goto drain;
+      const int sq = q_it % C::NQ, so = q_it % C::NO;
+      if (!wait_warp(br.q_full(sq), (q_it / C::NQ) & 1u, cx, SITE_QD_FULL)) goto drain;
       tc_fence_after();
-      issue_s(s);
+      issue_s(sq);
       commit(br.s_full());
-      issue_dp(s);
+      if (!wait_warp(br.do_full(so), (q_it / C::NO) & 1u, cx, SITE_QD_FULL)) goto drain;
+      tc_fence_after();
+      issue_dp(so);
       commit(br.dp_full());
     }
     for (int idx = 0; idx < n; ++idx) {
       const bool more = idx + 1 < n;
-      const int s = q_it % C::NS;
-      const int s1 = (q_it + 1) % C::NS;
-      if (!wait_warp(br.p_full(), step & 1u, cx, SITE_P_FULL)) goto drain;
+      const int sq = q_it % C::NQ, so = q_it % C::NO;
+      const int sq1 = (q_it + 1) % C::NQ, so1 = (q_it + 1) % C::NO;
+      if (more) {
+        // S^T of the next query tile as soon as the softmax has read this
+        // one: P^T and dS^T go to the dP^T columns, so the S^T columns are
+        // free from then on and S^T(i+1) overlaps the exponentials of step i
+        if (!wait_warp(br.s_free(), step & 1u, cx, SITE_S_FREE)) goto drain;
+        if (!wait_warp(br.q_full(sq1), ((q_it + 1) / C::NQ) & 1u, cx, SITE_QD_FULL)) goto drain;
+        tc_fence_after();
+        issue_s(sq1);
+        commit(br.s_full());
+      }
+      if (!wait_warp(br.pd_full(), step & 1u, cx, SITE_DS_FULL)) goto drain;
       if (idx == 0 && units > 0 &&
           !wait_warp(br.acc_free(), (units - 1) & 1u, cx, SITE_ACC_FREE))
         goto drain;
       tc_fence_after();
-      // dV += P^T dO (dO MN-major)
-      mma_tmem_a_split(t_dv, t_s, stmn_lo + ((s * 2 * C::TILE + C::TILE) >> 4), mn_hi, IDESC_ACC,
-                 idx > 0 ? 1u : 0u);
+      // dV += P^T dO (dO MN-major), P^T pairs at dP^T columns 0-31 / 64-95
+      mma_tmem_a_split(t_dv, t_dp, domn_lo + ((so * C::TILE) >> 4), mn_hi, IDESC_ACC,
+                       idx > 0 ? 1u : 0u);
+      commit(br.do_empty(so));
+      // dK += dS^T Q (Q MN-major), dS^T pairs at dP^T columns 32-63 / 96-127
+      mma_tmem_a_split(t_dk, t_dp + 32, qmn_lo + ((sq * C::TILE) >> 4), mn_hi, IDESC_ACC,
+                       idx > 0 ? 1u : 0u);
+      commit(br.q_empty(sq));
       if (more) {
-        // S^T of the next step may overwrite P^T: the tensor pipe runs the
-        // MMAs in order, so dV has read it by then
-        if (!wait_warp(br.qd_full(s1), ((q_it + 1) / C::NS) & 1u, cx, SITE_QD_FULL)) goto drain;
+        // dP^T of the next tile overwrites P^T and dS^T after dV and dK have
+        // read them (in-order tensor pipe)
+        if (!wait_warp(br.do_full(so1), ((q_it + 1) / C::NO) & 1u, cx, SITE_QD_FULL)) goto drain;
         tc_fence_after();
-        issue_s(s1);
-        commit(br.s_full());
-      }
-      if (!wait_warp(br.ds_full(), step & 1u, cx, SITE_DS_FULL)) goto drain;
-      tc_fence_after();
-      // dK += dS^T Q (Q MN-major)
-      mma_tmem_a_split(t_dk, t_dp, stmn_lo + ((s * 2 * C::TILE) >> 4), mn_hi, IDESC_ACC,
-                 idx > 0 ? 1u : 0u);
-      commit(br.qd_empty(s));
-      if (more) {
-        issue_dp(s1);
+        issue_dp(so1);
         commit(br.dp_full());
       }
       ++step;
@@ -886,8 +916,8 @@ drain:
 }
 
 template <int D>
-__device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, const float* vec_smem,
-                           int wg, const Ctl& cx) {
+__device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, const float* lse_smem,
+                           const float* dv_smem, int wg, const Ctl& cx) {
   using C = KCfg<D>;
   constexpr int D2 = D / 2;                        // dK, dV columns of this warpgroup
   const int t = threadIdx.x & 127;                 // key row inside the tile
@@ -907,22 +937,25 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
     QWalk it;
     it.start(p, x);
     for (int idx = 0; idx < x.n; ++idx, it.next(p)) {
-      const int s = q_it % C::NS;
+      const int sq = q_it % C::NQ, so = q_it % C::NO;
       // the diagonal tile of the own block: query column j sees key row t
       // only when j >= t (j > t under the strict mask)
       const bool diag = p.causal && it.i == x.jb && it.qt == x.kt;
       const int first = t + p.diag_shift - col0;   // first allowed local column
       if (!wait_warp(br.s_full(), step & 1u, cx, SITE_S_FULL)) return;
-      // the loader's -lse and D for this stage are visible once its phase
-      // completed (it completed before S^T was issued)
-      if (!wait_warp(br.qd_full(s), (q_it / C::NS) & 1u, cx, SITE_QD_FULL)) return;
+      // the loader's -lse of this Q stage is visible once its phase completed
+      // (it completed before S^T was issued)
+      if (!wait_warp(br.q_full(sq), (q_it / C::NQ) & 1u, cx, SITE_QD_FULL)) return;
       tc_fence_after();
-      const float* nl = vec_smem + s * 2 * TM + col0;
-      const float* dvv = vec_smem + s * 2 * TM + TM + col0;
+      const float* nl = lse_smem + sq * TM + col0;
+      const float* dvv = dv_smem + so * TM + col0;
       uint32_t sr[64];
       tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
+      // S^T is in registers: its columns may take the next tile's S^T
+      tc_fence_before();
+      mbar_arrive(br.s_free());
       uint32_t pk[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -944,31 +977,28 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
         }
         pk[j] = pack_bf16x2(p0, p1);
       }
-      // P^T as bf16 pairs over this warpgroup's own S^T columns
-      tmem_st32(t_s, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(br.p_full());
       if (!wait_warp(br.dp_full(), step & 1u, cx, SITE_DP_FULL)) return;
+      // D of this dO stage (its phase completed before dP^T was issued)
+      if (!wait_warp(br.do_full(so), (q_it / C::NO) & 1u, cx, SITE_QD_FULL)) return;
       tc_fence_after();
       {
-        // both 32-query chunks of dP^T are read before any dS^T pair
-        // overwrites them
+        // this warpgroup's 64 dP^T columns are read whole, then P^T (pairs,
+        // columns 0-31) and dS^T (pairs, columns 32-63) replace them
         uint32_t dp[2][32];
         tmem_ld32(t_dp, dp[0]);
         tmem_ld32(t_dp + 32, dp[1]);
         tmem_wait_ld();
+        uint32_t ds[32];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t ds[16];
+        for (int cc = 0; cc < 2; ++cc)
           ds_chunk<true>(*reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * cc]), dp[cc],
-                         dvv + 32 * cc, 0.f, ds);
-          tmem_st16(t_dp + 16 * cc, ds);
-        }
+                         dvv + 32 * cc, 0.f, *reinterpret_cast<uint32_t(*)[16]>(&ds[16 * cc]));
+        tmem_st32(t_dp, pk);
+        tmem_st32(t_dp + 32, ds);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(br.ds_full());
+      mbar_arrive(br.pd_full());
       ++step;
       ++q_it;
     }
@@ -997,25 +1027,35 @@ template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   using C = KCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gen = smem_raw + (base - raw);
-  float* vec_smem = reinterpret_cast<float*>(gen + C::OFF_VEC);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gen + C::OFF_MISC);
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gen + C::OFF_MISC + 4);
-  const KBars br{base + C::OFF_BAR, C::NS};
+  const uint32_t base = smem_u32(smem_raw);
+  if (base & 1023u) {
+    // the layout has no alignment slack (see KCfg); never seen on B200
+    if (threadIdx.x == 0)
+      atomicCAS(&g_status, 0ull, (static_cast<unsigned long long>(RA_ERR_UNSUPPORTED) << 32) |
+                                     (0xFFFFull << 16) | (blockIdx.x & 0xFFFF));
+    return;
+  }
+  float* lse_smem = reinterpret_cast<float*>(smem_raw + C::OFF_LSE);
+  float* dv_smem = reinterpret_cast<float*>(smem_raw + C::OFF_DV);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem_raw + C::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem_raw + C::OFF_MISC + 4);
+  const KBars br{base + C::OFF_BAR, C::NQ, C::NO};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     mbar_init(br.kv_full(), 1);
     mbar_init(br.kv_empty(), 1);
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(br.qd_full(s), 1 + 32);   // TMA transaction arrive + 32 loader lanes
-      mbar_init(br.qd_empty(s), 1);
+    for (int s = 0; s < C::NQ; ++s) {
+      mbar_init(br.q_full(s), 1 + 32);    // TMA transaction arrive + 32 loader lanes
+      mbar_init(br.q_empty(s), 1);
+    }
+    for (int s = 0; s < C::NO; ++s) {
+      mbar_init(br.do_full(s), 1 + 32);
+      mbar_init(br.do_empty(s), 1);
     }
     mbar_init(br.s_full(), 1);
     mbar_init(br.dp_full(), 1);
-    mbar_init(br.p_full(), SOFTMAX_THREADS);
-    mbar_init(br.ds_full(), SOFTMAX_THREADS);
+    mbar_init(br.s_free(), SOFTMAX_THREADS);
+    mbar_init(br.pd_full(), SOFTMAX_THREADS);
     mbar_init(br.acc_done(), 1);
     mbar_init(br.acc_free(), SOFTMAX_THREADS);
     mbar_init(br.drain(), 1);
@@ -1038,9 +1078,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __gri
   const uint32_t tmem = *tmem_holder;
   const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
   if (warp < 8) {
-    kv_softmax<D>(p, br, tmem, vec_smem, warp >> 2, cx);
+    kv_softmax<D>(p, br, tmem, lse_smem, dv_smem, warp >> 2, cx);
   } else if (warp == WARP_LOAD) {
-    kv_loader<D>(p, br, base, vec_smem, cx);
+    kv_loader<D>(p, br, base, lse_smem, dv_smem, cx);
   } else {
     kv_mma<D>(p, br, base, tmem, cx);
   }
