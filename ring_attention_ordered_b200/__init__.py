@@ -1,10 +1,12 @@
 """B200-native ring-ordered blockwise attention.
 
 The product is the C-ABI library ``libring_attn.so`` (kernels for sm_100a,
-declared in ``include/ring_attn.h``).  This package holds its sources
-(``csrc/``), the in-tree build (``build``), the ctypes binding (``_lib``), a
-torch-facing wrapper (``api``) that only marshals tensors into the C calls,
-and the seeded synthetic inputs (``inputs``).
+declared in ``include/ring_attn.h``: forward, backward, their per-visit forms
+and the log-sum-exp merge).  This package holds its sources (``csrc/``), the
+in-tree build (``build``), the ctypes binding (``_lib``), a torch-facing
+wrapper (``api``) that only marshals tensors into the C calls, the
+multi-process ring over torch.distributed with its contiguous, zigzag and
+striped layouts (``ring``), and the seeded synthetic inputs (``inputs``).
 """
 
 from ._lib import (  # noqa: F401
