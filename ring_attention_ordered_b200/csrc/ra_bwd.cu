@@ -16,18 +16,23 @@
 // which dK_j, dV_j would travel the ring; causal visits with a later K/V block
 // are skipped (L4 §4.5 limitation 2).
 //
-// How (B200 design): two persistent kernels, one CTA per SM, each with one
-// softmax warpgroup (warps 0-3, one TMEM lane = one tile row), a TMA loader
-// warp (4) and a tcgen05.mma warp (5).
+// How (B200 design): two persistent kernels, one CTA per SM, each with two
+// softmax warpgroups (warps 0-7; both cover all 128 TMEM lanes, one tile row
+// per lane, and split the tile's 128 columns), a TMA loader warp (8) and a
+// tcgen05.mma warp (9).
 //   * ra_bwd_dq_kernel: a unit is one 128-row query tile of one head; it
 //     computes D for its rows (written to the workspace), then for every K/V
 //     tile S = Q K^T and dP = dO V^T into TMEM, P and dS in the softmax
-//     warps (dS as bf16 over dP), and dQ += dS K accumulated in TMEM.
+//     warps (dS as bf16 over dP), and dQ += dS K accumulated in TMEM.  S is
+//     released as soon as it is read, so the next tile's S overlaps the
+//     exponentials; K (read early by S and late by dQ) has three stages.
 //   * ra_bwd_dkdv_kernel (after it, on the same stream): a unit is one
 //     128-key tile of one K/V head; for every query tile of every head of the
-//     group, S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T in the
-//     softmax warps (bf16, over S^T and dP^T), dV += P^T dO and dK += dS^T Q
-//     accumulated in TMEM: no atomics, every gradient is written once.
+//     group, S^T = K Q^T and dP^T = V dO^T into TMEM; the softmax warps read
+//     S^T (released at once, so the next tile's S^T overlaps them), form P^T,
+//     read dP^T and write P^T and dS^T as bf16 over it; dV += P^T dO and
+//     dK += dS^T Q accumulate in TMEM: no atomics, every gradient is written
+//     once.  Q (read early by S^T and late by dK) has three stages.
 //   P is rounded to bf16 once and that value feeds both dV and dS.
 //   Every mbarrier wait is bounded (ra_sync.cuh).
 #include <cuda.h>
