@@ -215,3 +215,31 @@ def merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torc
 def check_status(stream=None):
     with torch.cuda.device(torch.cuda.current_device()):
         _lib.ring_attn_check_status(_stream_handle(stream))
+
+
+class _RingAttention(torch.autograd.Function):
+    """Autograd bridge: forward through ring_attn_fwd (saving out and lse),
+    backward through ring_attn_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, n_ring, causal, scale):
+        out, lse = fwd(q, k, v, n_ring, causal, scale)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.n_ring, ctx.causal, ctx.scale = n_ring, causal, scale
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = bwd(q, k, v, out, dout.contiguous().to(torch.bfloat16), lse, ctx.n_ring,
+                         ctx.causal, ctx.scale)
+        return dq, dk, dv, None, None, None
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: bool,
+              scale: float | None = None) -> torch.Tensor:
+    """Differentiable ring-ordered attention on one GPU: the output of
+    ``fwd``, with gradients for q, k and v from ``bwd``."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    return _RingAttention.apply(q, k, v, n_ring, causal, scale)

@@ -429,3 +429,33 @@ def ring_attention_bwd_emulated(q, k, v, out, dout, lse, world: int, causal: boo
     dk = unshard([finish(acc[h][0], hosts[h]["k"]) for h in range(world)], layout)
     dv = unshard([finish(acc[h][1], hosts[h]["v"]) for h in range(world)], layout)
     return dq, dk, dv
+
+
+class RingAttentionFn(torch.autograd.Function):
+    """Autograd bridge for the multi-process ring: forward by
+    ``ring_attention``, backward by ``ring_attention_bwd`` (same layout,
+    group and visits)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale, layout, group, visit, bwd_visit, finish):
+        out, lse = ring_attention(q, k, v, causal, scale, layout, group, visit)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.args = (causal, scale, layout, group, bwd_visit, finish)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        causal, scale, layout, group, bwd_visit, finish = ctx.args
+        dq, dk, dv = ring_attention_bwd(q, k, v, out, dout.contiguous().to(out.dtype), lse,
+                                        causal, scale, layout, group, bwd_visit, finish)
+        return dq, dk, dv, None, None, None, None, None, None, None
+
+
+def ring_attention_fn(q, k, v, causal: bool, scale: float | None = None,
+                      layout: str = "contiguous", group=None, visit=None, bwd_visit=None,
+                      finish=None):
+    """Differentiable ``ring_attention``: this host's output, with gradients
+    for its q, k and v through the backward ring."""
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    return RingAttentionFn.apply(q, k, v, causal, scale, layout, group, visit, bwd_visit, finish)
