@@ -179,7 +179,6 @@ def test_bwd_large_workloads_dq_rows(ra, name, n_sample):
 def test_autograd_function_matches_oracle(ra):
     """api.attention under torch.autograd: output and q, k, v gradients of a
     GQA causal problem against the oracle."""
-    from parity import compare
     from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
     q, k, v = make_inputs(1, 4, 2, 768, 128, seed=61)
     do = make_grad_output(1, 768, 4, 128, seed=61)
