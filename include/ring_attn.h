@@ -8,8 +8,10 @@
  * (i - t) mod n_ring for t = 0..n_ring-1 (L3 definition, L4 §4.2); every
  * visit is exact blockwise attention whose partial result is folded into a
  * running online-softmax accumulator (L4 §4.3), and under causal masking the
- * later blocks are skipped (L4 §4.5, limitation 2).  The n_ring hosts are
- * emulated as n_ring sequence blocks on one GPU; no data leaves the device.
+ * later blocks are skipped (L4 §4.5, limitation 2).  ring_attn_fwd and
+ * ring_attn_bwd emulate the n_ring hosts as n_ring sequence blocks on one GPU;
+ * ring_attn_fwd_visit and ring_attn_bwd_visit are one host's step of a ring
+ * spread over devices, whose exchange the caller performs.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -19,9 +21,10 @@
  *     launched; device-side failures are reported by ring_attn_check_status.
  *   - No C++ exception crosses the ABI.  A non-OK status leaves a one-line
  *     explanation that ring_attn_last_error() returns (per host thread).
- *   - The library holds no device allocation of its own except two status
- *     words per device (static device variables of the module: one for the
- *     forward kernels, one for the backward kernels).
+ *   - The library holds no device allocation of its own except static
+ *     device variables of the module: two status words per device (forward
+ *     and backward kernels) and the fixed 4 MiB array of
+ *     ring_attn_bwd_noalloc.
  */
 #ifndef RING_ATTN_H_
 #define RING_ATTN_H_
