@@ -65,12 +65,17 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// Query SM count and compute capability of the current device once.
+// Query SM count and compute capability of the current device once.  Also
+// makes the device's primary context current on the calling thread: a thread
+// that has only been told its device (such as torch's autograd worker) may
+// have none yet, and the tensor-map encoder needs one.
 ra_status device_info(int* sms) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(RA_ERR_UNSUPPORTED, "device index %d", dev);
+  if ((e = cudaSetDevice(dev)) != cudaSuccess)
+    return fail(RA_ERR_CUDA, "cudaSetDevice: %s", cudaGetErrorString(e));
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_cc_ok[dev] == 0) {
     int major = 0, minor = 0, n = 0;
