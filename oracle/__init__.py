@@ -18,9 +18,12 @@ are
 
 ``attn_fp64`` holds the forward pass and the ring; ``attn_bwd_fp64`` the
 gradients of the same definition (the backward pass the FlashAttention
-article's recomputation serves).
+article's recomputation serves); ``fp8_fp64`` the E4M3 format, the block
+quantisation of the FP8 forward (FlashAttention article, FlashAttention-3)
+and the attention of the dequantised tensors.
 
-Every function here has a pin in ``tests/test_oracle.py`` against something
+Every function here has a pin in ``tests/test_oracle.py``,
+``tests/test_oracle_bwd.py`` or ``tests/test_oracle_fp8.py`` against something
 other than itself (a library routine, a closed form, an invariant, the pages'
 worked example, or brute force on tiny inputs); none is parity unpinned.
 """
@@ -45,4 +48,14 @@ from .attn_bwd_fp64 import (  # noqa: F401
     attention_bwd_dq_rows,
     attention_bwd_kv_rows,
     block_attention_bwd,
+)
+from .fp8_fp64 import (  # noqa: F401
+    E4M3_MAX,
+    DequantView,
+    attention_fp8,
+    attention_fp8_rows,
+    dequantize_blocks,
+    e4m3_decode,
+    e4m3_encode,
+    quantize_blocks,
 )
