@@ -113,7 +113,8 @@ KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd.cu",
                   "ring_attention_ordered_b200/csrc/ra_internal.h",
                   "ring_attention_ordered_b200/csrc/ra_merge_math.cuh",
                   "ring_attention_ordered_b200/csrc/ra_sync.cuh",
-                  "ring_attention_ordered_b200/csrc/ra_exp2.cuh"]
+                  "ring_attention_ordered_b200/csrc/ra_exp2.cuh",
+                  "ring_attention_ordered_b200/csrc/ra_schedule.cuh"]
 TRAFFIC_RECORD = "profiles/ra_fwd_l128k_h32_causal_dram.md"
 
 
@@ -216,6 +217,71 @@ def run_reference(args, w, world, rank):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def fp8_supported(w) -> bool:
+    return w.d == 128 and (w.L // w.n_ring) % 128 == 0
+
+
+def time_fp8(api, q, k, v, w, stream, steps: int, peaks: dict, world: int = 1, dev=None):
+    """The FP8 forward on the workload's inputs: block quantisation of q, k, v
+    (timed on its own, HBM-bound: 2 bytes read + 1 byte written per element
+    plus the scales) and W = 2 warm-up then ``steps`` timed ring_attn_fwd_fp8
+    launches.  Returns a dict for the JSON line."""
+    import torch
+    q8, sq = api.quantize_fp8(q, stream=stream)
+    k8, sk = api.quantize_fp8(k, stream=stream)
+    v8, sv = api.quantize_fp8(v, stream=stream)
+    out8 = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    lse8 = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=q.device)
+
+    def quant():
+        api.quantize_fp8(q, q8, sq, stream=stream)
+        api.quantize_fp8(k, k8, sk, stream=stream)
+        api.quantize_fp8(v, v8, sv, stream=stream)
+
+    def fwd8():
+        api.fwd_fp8(q8, sq, k8, sk, v8, sv, w.n_ring, w.causal, w.scale, out=out8, lse=lse8,
+                    stream=stream)
+
+    for _ in range(2):
+        quant()
+        fwd8()
+    api.check_status(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    qreps = 5
+    e0.record(stream)
+    for _ in range(qreps):
+        quant()
+    e1.record(stream)
+    torch.cuda.synchronize(q.device)
+    q_ms = e0.elapsed_time(e1) / qreps
+    e0.record(stream)
+    for _ in range(steps):
+        fwd8()
+    e1.record(stream)
+    torch.cuda.synchronize(q.device)
+    api.check_status(stream)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    flops = w.flops()
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = 2.0 * peaks["bf16_tflops_sustained"]
+    qbytes = 3 * (q.numel() + k.numel() + v.numel()) + 4 * (sq.numel() + sk.numel() + sv.numel())
+    return {
+        "ms": ms, "TFLOP/s": world * achieved, "steps": steps, "launches_per_call": 1,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None, "kernel": "ra_fwd_fp8_kernel",
+                     "peak_kind": "E4M3 dense = 2 x bf16_tflops_sustained "
+                                  f"({peaks['source']}), the nominal 4.5 / 2.25 PFLOP/s ratio"},
+        "frac_of_bf16_sustained": achieved / peaks["bf16_tflops_sustained"],
+        "quantize": {"ms": q_ms, "GB/s": qbytes / (q_ms / 1e3) / 1e9,
+                     "frac_hbm": qbytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "bytes": qbytes, "launches": 3},
+        "ms_with_quantize": ms + q_ms,
+        "tolerance": "vs exact attention of the dequantised inputs: per element "
+                     "sum_c (2^-4 w_c + 2^-10 / (f_c l_M)) |v_c| + 2^-9 |O| + 1e-3 sum_c w_c |v_c|; "
+                     "lse 1e-3",
+    }
 
 
 def run_ours(args, w, world, rank, local):
@@ -394,6 +460,14 @@ def run_ours(args, w, world, rank, local):
                                   "execute 3.5 x forward (S and dP are recomputed for dQ)"}
         del do, dq, dk, dv, ws
 
+    # the FP8 forward on the same workload (its own line object; the headline
+    # value is the bf16 forward above)
+    fp8 = None
+    if not args.no_fp8 and fp8_supported(w):
+        if world > 1:
+            dist.barrier()
+        fp8 = time_fp8(api, q, k, v, w, stream, max(3, min(args.steps, 10)), peaks, world, dev)
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -441,6 +515,7 @@ def run_ours(args, w, world, rank, local):
         "gpu_launches": args.steps,
         "clocks": clocks,
         "bwd": bwd,
+        "fp8": fp8,
         "merge": {"ms": merge_ms, "GB/s": merge_bytes / (merge_ms / 1e3) / 1e9,
                   "frac_hbm": merge_bytes / (merge_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                   "rows": rows, "d": w.d},
@@ -512,7 +587,12 @@ def run_all_workloads(args):
             "kind": "workload_bwd", "workload": w.describe(), "name": name, "steps": bsteps,
             "ms": bms, "TFLOP/s": btf, "frac_of_burst": btf / peaks["bf16_tflops"],
             "flop_convention": "2.5 x forward"}), flush=True)
-        del q, k, v, out, lse, do, dq, dk, dv, ws
+        del do, dq, dk, dv, ws
+        if fp8_supported(w):
+            f8 = time_fp8(api, q, k, v, w, stream, max(2, steps // 2), peaks)
+            print(json.dumps({"kind": "workload_fp8", "workload": w.describe(), "name": name,
+                              **f8}), flush=True)
+        del q, k, v, out, lse
         torch.cuda.empty_cache()
     return 0
 
@@ -669,6 +749,7 @@ def main():
     ap.add_argument("--workload", default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass leg")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward leg")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--all-workloads", action="store_true",
                     help="print one line per named workload instead of the benchmark line")

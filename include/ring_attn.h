@@ -22,9 +22,9 @@
  *   - No C++ exception crosses the ABI.  A non-OK status leaves a one-line
  *     explanation that ring_attn_last_error() returns (per host thread).
  *   - The library holds no device allocation of its own except static
- *     device variables of the module: two status words per device (forward
- *     and backward kernels) and the fixed 4 MiB array of
- *     ring_attn_bwd_noalloc.
+ *     device variables of the module: three status words per device (bf16
+ *     forward, backward and FP8 forward kernels) and the fixed 4 MiB array
+ *     of ring_attn_bwd_noalloc.
  */
 #ifndef RING_ATTN_H_
 #define RING_ATTN_H_
@@ -278,9 +278,60 @@ ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b
                           ra_stream_t stream);
 
 /*
+ * ring_attn_quantize_fp8 -- block quantisation of a bf16 tensor to E4M3 for
+ * ring_attn_fwd_fp8 (the FP8 forward of the FlashAttention article,
+ * developer.aliyun page, section 二, FlashAttention-3: FP8 GEMMs with block
+ * quantisation).  A block is the 128-row tile of one (batch, head):
+ *     scale[b, h, t] = amax / 448 in float32 (1 if the tile is all zeros),
+ *                      amax over rows [128t, 128t + 128) and all d columns;
+ *     codes[b, r, h, c] = E4M3(x[b, r, h, c] / scale), the quotient rounded
+ *                      to float32, then to E4M3 (OCP 8-bit format: bias 7,
+ *                      largest finite 448, no infinities) with ties to even,
+ *                      magnitudes above 448 saturated.
+ * When L is not a multiple of 128 the last tile holds the remaining rows.
+ *
+ *   x       bf16 [B, L, H, d], contiguous, 16-byte aligned, finite values
+ *   codes   uint8 [B, L, H, d] (E4M3 bit patterns), 16-byte aligned
+ *   scales  fp32 [B, H, ceil(L / 128)], 4-byte aligned
+ *   d a multiple of 8 in [8, 256]; B, H <= 65535.  Outputs must not overlap x
+ *   or each other.  B*H*L == 0 launches nothing.
+ * Errors: RA_ERR_INVALID_ARG for negative sizes, null, misaligned or
+ * overlapping pointers; RA_ERR_UNSUPPORTED for other d or B, H above 65535.
+ */
+ra_status ring_attn_quantize_fp8(const void* x, void* codes, float* scales, int B, int64_t L,
+                                 int H, int d, ra_stream_t stream);
+
+/*
+ * ring_attn_fwd_fp8 -- the ring-ordered forward of ring_attn_fwd (same
+ * blocks, ring order, causal skipping and masking, GQA mapping and lse
+ * convention) computed from block-quantised E4M3 inputs: both GEMMs on the
+ * FP8 tensor cores, scores scaled by scale * sq * sk per tile pair, fp32
+ * softmax statistics, the probabilities rounded to E4M3 before the P V
+ * product, bf16 output.  It approximates exact attention of the dequantised
+ * tensors code * scale; the error is that of E4M3 probabilities (relative
+ * 2^-4 per weight, absolute 2^-10 below E4M3's normal range).
+ *
+ *   q8            uint8 [B, L, Hq, 128]  E4M3 codes (ring_attn_quantize_fp8)
+ *   k8, v8        uint8 [B, L, Hkv, 128]
+ *   sq            fp32 [B, Hq, L / 128]  tile scales, finite and > 0
+ *   sk, sv        fp32 [B, Hkv, L / 128]
+ *   out           bf16 [B, L, Hq, 128]
+ *   lse           fp32 [B, Hq, L], natural log
+ *   d must be 128 and L / n_ring a multiple of 128 (else RA_ERR_UNSUPPORTED);
+ *   the other sizes, values and errors are those of ring_attn_fwd.  All
+ *   pointers 16-byte aligned; outputs must not overlap the inputs or each
+ *   other.
+ */
+ra_status ring_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                            const float* sk, const float* sv, void* out, float* lse, int B, int Hq,
+                            int Hkv, int64_t L, int d, int n_ring, int causal, float scale,
+                            ra_stream_t stream);
+
+/*
  * ring_attn_check_status -- synchronise `stream`, then read and clear the
  * device status words of the current device.  Every device-side wait of the
- * forward and backward kernels is bounded (see ring_attn_set_wait_limit_ns); a wait that
+ * forward (bf16 and FP8) and backward kernels is bounded (see
+ * ring_attn_set_wait_limit_ns); a wait that
  * runs out makes the kernel record RA_ERR_TIMEOUT, release its tensor memory
  * and return, leaving the CUDA context usable.  Returns RA_ERR_CUDA if the
  * synchronisation itself fails.
@@ -291,7 +342,7 @@ ra_status ring_attn_check_status(ra_stream_t stream);
  * (nanoseconds; default 5e9).  0 restores the default.  Process-wide. */
 ra_status ring_attn_set_wait_limit_ns(uint64_t ns);
 
-/* Cap on the number of persistent CTAs of the forward kernel (0 = one per
+/* Cap on the number of persistent CTAs of the forward kernels (0 = one per
  * SM, the default).  Process-wide; used to exercise the scheduler. */
 ra_status ring_attn_set_max_ctas(int n);
 
@@ -308,7 +359,8 @@ enum { RA_SCHEDULE_AUTO = 0, RA_SCHEDULE_LONGEST_FIRST = 1, RA_SCHEDULE_HEAD_MAJ
 ra_status ring_attn_set_schedule(int schedule);
 
 /* Host-side fault injection for tests.  Bit 0: the loader of the forward
- * kernel and of the backward dQ kernel skips its first query-tile load, so
+ * kernels (bf16 and FP8) and of the backward dQ kernel skips its first
+ * query-tile load, so
  * the first bounded wait on it runs out and the call reports RA_ERR_TIMEOUT
  * through ring_attn_check_status.  0 clears.  Process-wide. */
 ra_status ring_attn_debug_inject(unsigned flags);

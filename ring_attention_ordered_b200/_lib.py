@@ -33,6 +33,9 @@ SIGNATURES = {
     "ring_attn_round_bf16": (_I, [_P, _P, _I64, _P]),
     "ring_attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I,
                                    ctypes.c_float, _P]),
+    "ring_attn_quantize_fp8": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P]),
+    "ring_attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I,
+                               ctypes.c_float, _P]),
     "ring_attn_merge": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I, _P]),
     "ring_attn_check_status": (_I, [_P]),
     "ring_attn_set_wait_limit_ns": (_I, [ctypes.c_uint64]),
@@ -126,6 +129,16 @@ def ring_attn_fwd_visit(q, k, v, o_acc, lse_acc, out, B, Hq, Hkv, l, d, diag, fo
                         stream=0):
     return _check(load().ring_attn_fwd_visit(q, k, v, o_acc, lse_acc, out, B, Hq, Hkv, l, d,
                                              int(diag), int(fold), float(scale), stream))
+
+
+def ring_attn_quantize_fp8(x, codes, scales, B, L, H, d, stream=0):
+    return _check(load().ring_attn_quantize_fp8(x, codes, scales, B, L, H, d, stream))
+
+
+def ring_attn_fwd_fp8(q8, k8, v8, sq, sk, sv, out, lse, B, Hq, Hkv, L, d, n_ring, causal, scale,
+                      stream=0):
+    return _check(load().ring_attn_fwd_fp8(q8, k8, v8, sq, sk, sv, out, lse, B, Hq, Hkv, L, d,
+                                           n_ring, int(bool(causal)), float(scale), stream))
 
 
 def ring_attn_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d, stream=0):

@@ -194,6 +194,61 @@ def fwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Te
     return o_acc, lse_acc, out
 
 
+def quantize_fp8(x: torch.Tensor, codes: torch.Tensor | None = None,
+                 scales: torch.Tensor | None = None, stream=None):
+    """Block quantisation of x bf16 [B, L, H, d] to E4M3: returns (codes
+    uint8 [B, L, H, d], scales fp32 [B, H, ceil(L / 128)]), one scale per
+    128-row tile of each (batch, head).  The codes are raw E4M3 bit patterns
+    (``codes.view(torch.float8_e4m3fn)`` reads them as FP8)."""
+    _check_cuda(x, "x", torch.bfloat16, 4)
+    B, L, H, d = x.shape
+    if codes is None:
+        codes = torch.empty((B, L, H, d), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, (L + 127) // 128), dtype=torch.float32, device=x.device)
+    _check_cuda(codes, "codes", torch.uint8, 4)
+    _check_cuda(scales, "scales", torch.float32, 3)
+    with torch.cuda.device(x.device):
+        _lib.ring_attn_quantize_fp8(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), B, L, H, d,
+                                    _stream_handle(stream))
+    return codes, scales
+
+
+def fwd_fp8(q8: torch.Tensor, sq: torch.Tensor, k8: torch.Tensor, sk: torch.Tensor,
+            v8: torch.Tensor, sv: torch.Tensor, n_ring: int, causal: bool,
+            scale: float | None = None, out: torch.Tensor | None = None,
+            lse: torch.Tensor | None = None, stream=None):
+    """Ring-ordered attention forward on FP8 inputs from ``quantize_fp8``:
+    q8 [B, L, Hq, 128] with sq [B, Hq, L/128], k8/v8 [B, L, Hkv, 128] with
+    sk/sv [B, Hkv, L/128].  Returns (out bf16 [B, L, Hq, 128], lse fp32
+    [B, Hq, L]).  ``scale`` defaults to 1/sqrt(d)."""
+    for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _check_cuda(t, n, torch.uint8, 4)
+    for t, n in ((sq, "sq"), (sk, "sk"), (sv, "sv")):
+        _check_cuda(t, n, torch.float32, 3)
+    B, L, Hq, d = q8.shape
+    Hkv = k8.shape[2]
+    if k8.shape != (B, L, Hkv, d) or v8.shape != k8.shape:
+        raise ValueError(f"k8/v8 shape {tuple(k8.shape)}/{tuple(v8.shape)} does not match "
+                         f"q8 {tuple(q8.shape)}")
+    T = L // 128
+    if sq.shape != (B, Hq, T) or sk.shape != (B, Hkv, T) or sv.shape != (B, Hkv, T):
+        raise ValueError("scale tensors must be [B, H, L/128]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, L, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q8.device)
+    _check_cuda(out, "out", torch.bfloat16, 4)
+    _check_cuda(lse, "lse", torch.float32, 3)
+    with torch.cuda.device(q8.device):
+        _lib.ring_attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), sq.data_ptr(),
+                               sk.data_ptr(), sv.data_ptr(), out.data_ptr(), lse.data_ptr(), B,
+                               Hq, Hkv, L, d, n_ring, causal, scale, _stream_handle(stream))
+    return out, lse
+
+
 def merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,
           out: torch.Tensor | None = None, lse_out: torch.Tensor | None = None, stream=None):
     """Log-sum-exp merge of two partials: o [rows, d] fp32, lse [rows] fp32."""

@@ -199,6 +199,42 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_
       : "memory");
 }
 
+// The same two forms for kind::f8f6f4 (8-bit A and B, f32 accumulate; the
+// element types are named in the instruction descriptor).  K is 32 elements
+// (32 bytes) per instruction; an 8-bit A operand in tensor memory packs four
+// consecutive K elements into each 32-bit column.
+template <uint32_t A_OFF, uint32_t B_OFF>
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                          uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 al, bl;\n\t.reg .b64 da, db;\n\t"
+      "add.u32 al, %1, %7;\n\t"
+      "add.u32 bl, %3, %8;\n\t"
+      "mov.b64 da, {al, %2};\n\t"
+      "mov.b64 db, {bl, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %5, p;\n\t}"
+      :: "r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate),
+         "n"(A_OFF), "n"(B_OFF)
+      : "memory");
+}
+
+template <uint32_t A_COL, uint32_t B_OFF>
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                          uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 ta, bl;\n\t.reg .b64 db;\n\t"
+      "add.u32 ta, %1, %6;\n\t"
+      "add.u32 bl, %2, %7;\n\t"
+      "mov.b64 db, {bl, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [ta], db, %4, p;\n\t}"
+      :: "r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate),
+         "n"(A_COL), "n"(B_OFF)
+      : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05 operation the issuing thread
 // started so far has completed; executed only where `issue` is non-zero.
 __device__ __forceinline__ void tc_commit_if(uint32_t bar, uint32_t issue) {
@@ -282,6 +318,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
        | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0
+// in both fields), f32 accumulator.  b_mn_major selects an MN-major B.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4)                       // D format: f32
+       | (0u << 7)                       // A format: E4M3
+       | (0u << 10)                      // B format: E4M3
+       | ((b_mn_major ? 1u : 0u) << 16)  // B major
+       | (static_cast<uint32_t>(N >> 3) << 17)
+       | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -323,6 +370,19 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Four fp32 values to E4M3 (round to nearest even, saturating to +-448),
+// packed with v0 in the lowest byte: the order of K elements in a 32-bit
+// tensor-memory column of an 8-bit A operand.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r) : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
   return r;
 }
 

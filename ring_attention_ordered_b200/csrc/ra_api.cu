@@ -110,6 +110,22 @@ ra_status make_map(CUtensorMap* map, const void* base, int H, long long rows, in
   return RA_OK;
 }
 
+// Tensor map over the E4M3 codes of a [B*L, H, 128] byte array: box
+// {128, 1, 128} (one 128-byte swizzle row per head row), 128-byte swizzle.
+ra_status make_map_e4m3(CUtensorMap* map, const void* base, int H, long long rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(H) * 128};
+  cuuint32_t box[3] = {128, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return RA_OK;
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
@@ -478,14 +494,114 @@ ra_status ring_attn_merge(const float* o_a, const float* lse_a, const float* o_b
   return ok();
 }
 
+ra_status ring_attn_quantize_fp8(const void* x, void* codes, float* scales, int B, int64_t L,
+                                 int H, int d, ra_stream_t stream) {
+  if (B < 0 || H < 0 || L < 0) return fail(RA_ERR_INVALID_ARG, "negative size");
+  if (d < 8 || d > 256 || d % 8 != 0)
+    return fail(RA_ERR_UNSUPPORTED, "head dim %d (supported: multiples of 8 up to 256)", d);
+  if (static_cast<long long>(B) * H * L == 0) return ok();
+  if (B > 65535 || H > 65535) return fail(RA_ERR_UNSUPPORTED, "B and H must be <= 65535");
+  if (!x || !codes || !scales) return fail(RA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return fail(RA_ERR_INVALID_ARG, "x and codes must be 16-byte aligned, scales 4-byte aligned");
+  const size_t n = static_cast<size_t>(B) * L * H * d;
+  const size_t ns = static_cast<size_t>(B) * H * ((L + 127) / 128) * 4;
+  if (overlaps(codes, n, x, 2 * n) || overlaps(scales, ns, x, 2 * n) || overlaps(scales, ns, codes, n))
+    return fail(RA_ERR_INVALID_ARG, "outputs overlap the input or each other");
+  int sms = 0;
+  ra_status st = device_info(&sms);
+  if (st != RA_OK) return st;
+  cudaError_t e = ra::launch_quantize_fp8(static_cast<const __nv_bfloat16*>(x),
+                                          static_cast<uint8_t*>(codes), scales, B, L, H, d,
+                                          reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "quantize launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+ra_status ring_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                            const float* sk, const float* sv, void* out, float* lse, int B, int Hq,
+                            int Hkv, int64_t L, int d, int n_ring, int causal, float scale,
+                            ra_stream_t stream) {
+  ra_status st = check_forward_shape(B, Hq, Hkv, L, d, n_ring, causal, scale);
+  if (st != RA_OK) return st;
+  if (d != 128) return fail(RA_ERR_UNSUPPORTED, "the FP8 forward supports head dim 128 (got %d)", d);
+  if ((L / n_ring) % 128 != 0)
+    return fail(RA_ERR_UNSUPPORTED, "the FP8 forward needs L / n_ring to be a multiple of 128");
+  if (static_cast<long long>(B) * Hq * L == 0) return ok();
+  if (!q8 || !k8 || !v8 || !sq || !sk || !sv || !out || !lse)
+    return fail(RA_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[8] = {q8, k8, v8, sq, sk, sv, out, lse};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return fail(RA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const long long T = L / 128;
+  const size_t nq = static_cast<size_t>(B) * L * Hq * 128;
+  const size_t nkv = static_cast<size_t>(B) * L * Hkv * 128;
+  const size_t nsq = static_cast<size_t>(B) * Hq * T * 4, nskv = static_cast<size_t>(B) * Hkv * T * 4;
+  const size_t no = 2 * nq, nl = static_cast<size_t>(B) * Hq * L * 4;
+  const void* ins[6] = {q8, k8, v8, sq, sk, sv};
+  const size_t in_n[6] = {nq, nkv, nkv, nsq, nskv, nskv};
+  for (int i = 0; i < 6; ++i)
+    if (overlaps(out, no, ins[i], in_n[i]) || overlaps(lse, nl, ins[i], in_n[i]))
+      return fail(RA_ERR_INVALID_ARG, "outputs overlap the inputs");
+  if (overlaps(out, no, lse, nl)) return fail(RA_ERR_INVALID_ARG, "out and lse overlap");
+
+  int sms = 0;
+  if ((st = device_info(&sms)) != RA_OK) return st;
+  ra::Fp8FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  const long long rows = static_cast<long long>(B) * L;
+  if ((st = make_map_e4m3(&prm.tm_q, q8, Hq, rows)) != RA_OK) return st;
+  if ((st = make_map_e4m3(&prm.tm_k, k8, Hkv, rows)) != RA_OK) return st;
+  if ((st = make_map_e4m3(&prm.tm_v, v8, Hkv, rows)) != RA_OK) return st;
+  prm.sq = sq;
+  prm.sk = sk;
+  prm.sv = sv;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.L = static_cast<int>(L);
+  prm.n_ring = n_ring;
+  prm.blk_len = static_cast<int>(L / n_ring);
+  prm.causal = causal;
+  prm.tiles_per_blk = prm.blk_len / 128;
+  prm.pair_heads = prm.group >= 2 ? 1 : 0;
+  prm.head_slots = (prm.group + 1) / 2;
+  prm.pairs_per_blk = (prm.tiles_per_blk + 1) / 2;
+  prm.n_tiles = static_cast<int>(T);
+  const long long units =
+      prm.pair_heads
+          ? static_cast<long long>(B) * Hkv * prm.head_slots * n_ring * prm.tiles_per_blk
+          : static_cast<long long>(B) * Hq * n_ring * prm.pairs_per_blk;
+  if (units >= (1ll << 31)) return fail(RA_ERR_INVALID_ARG, "problem too large (%lld work units)", units);
+  prm.total_units = static_cast<int>(units);
+  const int sched = g_schedule.load();
+  prm.head_major = sched == RA_SCHEDULE_HEAD_MAJOR ||
+                   (sched == RA_SCHEDULE_AUTO && 2.0 * static_cast<double>(nkv) > kHeadMajorKvBytes);
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.wait_limit_ns = g_wait_limit_ns.load();
+  prm.debug_flags = g_debug_flags.load();
+  long long grid = sms;
+  const int cap = g_max_ctas.load();
+  if (cap > 0 && cap < grid) grid = cap;
+  if (grid > prm.total_units) grid = prm.total_units;
+  cudaError_t e = ra::launch_fwd_fp8(prm, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "FP8 forward launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 ra_status ring_attn_check_status(ra_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
-  unsigned long long v = 0, vb = 0;
+  unsigned long long v = 0, vb = 0, v8 = 0;
   e = ra::read_and_clear_status(&v);
   if (e == cudaSuccess) e = ra::read_and_clear_bwd_status(&vb);
+  if (e == cudaSuccess) e = ra::read_and_clear_fp8_status(&v8);
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
   if (v == 0) v = vb;
+  if (v == 0) v = v8;
   if (v == 0) return ok();
   const unsigned code = static_cast<unsigned>(v >> 32);
   const unsigned site = static_cast<unsigned>((v >> 16) & 0xFFFF);
@@ -531,6 +647,6 @@ const char* ring_attn_status_string(ra_status s) {
 
 const char* ring_attn_last_error(void) { return g_last_error.c_str(); }
 
-int ring_attn_version(void) { return 103; }
+int ring_attn_version(void) { return 104; }
 
 }  // extern "C"

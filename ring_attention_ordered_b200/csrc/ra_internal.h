@@ -40,6 +40,35 @@ struct FwdParams {
   unsigned debug_flags;
 };
 
+// Parameters of one FP8 forward launch (d = 128).  The tensor maps describe
+// the E4M3 codes of q, k and v as 3-D byte arrays {128, H, B*L} with a box of
+// {128, 1, 128}: one 128-byte swizzle row per head row, 128 consecutive rows
+// of one head.  sq [B, Hq, T], sk and sv [B, Hkv, T] hold the float32 scale
+// of each 128-row tile (T = L / 128).  The scheduling fields mean what they
+// mean in FwdParams.
+struct Fp8FwdParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  __nv_bfloat16* out;
+  float* lse;
+  int B, Hq, Hkv, group;
+  int L, blk_len, n_ring, causal;
+  int tiles_per_blk;
+  int pair_heads;
+  int head_slots;
+  int pairs_per_blk;
+  int total_units;
+  int head_major;
+  int n_tiles;         // T = L / 128
+  float scale_log2;    // scale * log2(e), before the per-tile scales
+  unsigned long long wait_limit_ns;
+  unsigned debug_flags;
+};
+
 // Parameters of the two backward launches (dQ kernel, then dK/dV kernel).
 // tm_q/tm_do view q and dout as {d, Hq, B*L}, tm_k/tm_v view k and v as
 // {d, Hkv, B*L}, with the forward's box and swizzle.
@@ -89,6 +118,12 @@ constexpr long long kNoAllocScratchRows = 1ll << 20;
 // Address of that scratch on the current device (looked up once per device).
 cudaError_t noalloc_scratch(void** ptr);
 cudaError_t read_and_clear_status(unsigned long long* out);
+
+cudaError_t launch_fwd_fp8(const Fp8FwdParams& prm, int grid, cudaStream_t stream);
+cudaError_t read_and_clear_fp8_status(unsigned long long* out);
+// Block quantisation of x bf16 [B, L, H, d] to E4M3 codes and per-tile scales.
+cudaError_t launch_quantize_fp8(const __nv_bfloat16* x, uint8_t* codes, float* scales, int B,
+                                long long L, int H, int d, cudaStream_t stream);
 
 cudaError_t launch_round_bf16(const float* src, __nv_bfloat16* dst, long long n, int num_sms,
                               cudaStream_t stream);

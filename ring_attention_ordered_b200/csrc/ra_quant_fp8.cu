@@ -1,0 +1,111 @@
+// Block quantisation to E4M3 for the FP8 forward (sm_100a).
+//
+// The FlashAttention article (developer.aliyun page, section 二,
+// FlashAttention-3 改进) keeps FP8 precision loss down by quantising in
+// blocks.  Here a block is the 128-row tile of one (batch, head): its scale is
+// amax / 448 in float32 (1 for an all-zero tile), and each element becomes
+// E4M3(x / scale), the quotient rounded to float32 (IEEE division) and then to
+// E4M3 with ties to even, saturating at +-448.  A ragged last tile holds the
+// remaining rows.
+//
+// One CTA per (tile, head, batch): 256 threads load the tile's rows (d bf16
+// values each, 16 bytes per load) into registers once, reduce |x| to the
+// tile's maximum, and write the codes (8 bytes per store) and the scale.  The
+// kernel is bound by HBM: 2 bytes read and 1 byte written per element.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ra_internal.h"
+
+namespace ra {
+namespace {
+
+constexpr int QT = 256;             // threads per CTA
+constexpr int ROWS = 128;           // rows per tile
+constexpr int MAX_CHUNKS = 16;      // 16-byte chunks per thread: 128 rows x 256 cols / 8 / 256
+
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float absmax8(uint4 v, float m) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(QT) ra_quant_fp8_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          uint8_t* __restrict__ codes,
+                                                          float* __restrict__ scales, long long L,
+                                                          int H, int d, int T) {
+  __shared__ float red[QT / 32];
+  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long long r0 = static_cast<long long>(t) * ROWS;
+  const int rows = static_cast<int>(min(static_cast<long long>(ROWS), L - r0));
+  const int cpr = d / 8;                         // 16-byte chunks per row
+  const int n = rows * cpr;
+  const long long row_stride = static_cast<long long>(H) * d;
+  const long long base = (static_cast<long long>(b) * L + r0) * row_stride + static_cast<long long>(h) * d;
+
+  uint4 v[MAX_CHUNKS];
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAX_CHUNKS; ++i) {
+    const int c = threadIdx.x + i * QT;
+    if (c < n) {
+      const int r = c / cpr, cc = c % cpr;
+      v[i] = __ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc);
+      m = absmax8(v[i], m);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float amax = red[0];
+#pragma unroll
+  for (int i = 1; i < QT / 32; ++i) amax = fmaxf(amax, red[i]);
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  if (threadIdx.x == 0) scales[(static_cast<long long>(b) * H + h) * T + t] = s;
+
+#pragma unroll
+  for (int i = 0; i < MAX_CHUNKS; ++i) {
+    const int c = threadIdx.x + i * QT;
+    if (c < n) {
+      const int r = c / cpr, cc = c % cpr;
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(hv[j]);
+        w[j] = e4m3x2(__fdiv_rn(f.x, s), __fdiv_rn(f.y, s));
+      }
+      uint2 out;
+      out.x = w[0] | (w[1] << 16);
+      out.y = w[2] | (w[3] << 16);
+      *(reinterpret_cast<uint2*>(codes + base + r * row_stride) + cc) = out;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_fp8(const __nv_bfloat16* x, uint8_t* codes, float* scales, int B,
+                                long long L, int H, int d, cudaStream_t stream) {
+  const long long T = (L + ROWS - 1) / ROWS;
+  if (T > 0x7fffffffll || H > 65535 || B > 65535) return cudaErrorInvalidValue;
+  if (d % 8 != 0 || d < 8 || d > 256) return cudaErrorInvalidValue;
+  dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>(H), static_cast<unsigned>(B));
+  ra_quant_fp8_kernel<<<grid, QT, 0, stream>>>(x, codes, scales, L, H, d, static_cast<int>(T));
+  return cudaGetLastError();
+}
+
+}  // namespace ra

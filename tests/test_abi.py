@@ -46,7 +46,7 @@ def test_status_strings_and_version(lib):
                                  "RA_ERR_CUDA", "RA_ERR_TIMEOUT"]):
         assert _lib.status_string(code) == name
     assert _lib.status_string(99) == "RA_ERR_UNKNOWN"
-    assert _lib.ring_attn_version() == 103
+    assert _lib.ring_attn_version() == 104
 
 
 # Fake, never-dereferenced device addresses: validation rejects these calls
@@ -256,3 +256,68 @@ def test_round_bf16_validation(lib):
     assert lib.ring_attn_round_bf16(DQ, DK, 12, None) == _lib.RA_ERR_INVALID_ARG      # n % 8
     assert lib.ring_attn_round_bf16(DQ + 4, DK, 16, None) == _lib.RA_ERR_INVALID_ARG  # alignment
     assert lib.ring_attn_round_bf16(DQ, DQ + 16, 16, None) == _lib.RA_ERR_INVALID_ARG  # overlap
+
+
+SQ, SK, SV = 7 * A * 64, 8 * A * 64, 9 * A * 64
+
+
+def fp8_status(lib, **kw):
+    args = dict(q8=Q, k8=K, v8=V, sq=SQ, sk=SK, sv=SV, out=O, lse=LSE, B=1, Hq=2, Hkv=2, L=512,
+                d=128, n_ring=4, causal=1, scale=0.088)
+    args.update(kw)
+    return lib.ring_attn_fwd_fp8(args["q8"], args["k8"], args["v8"], args["sq"], args["sk"],
+                                 args["sv"], args["out"], args["lse"], args["B"], args["Hq"],
+                                 args["Hkv"], args["L"], args["d"], args["n_ring"],
+                                 args["causal"], args["scale"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=64), _lib.RA_ERR_UNSUPPORTED),              # FP8 forward is d = 128 only
+    (dict(n_ring=8), _lib.RA_ERR_UNSUPPORTED),          # blocks of 64 rows
+    (dict(L=510), _lib.RA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), _lib.RA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.RA_ERR_INVALID_ARG),
+    (dict(causal=3), _lib.RA_ERR_INVALID_ARG),
+    (dict(sq=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(sk=SK + 4), _lib.RA_ERR_INVALID_ARG),         # not 16-byte aligned
+    (dict(out=Q + 4096), _lib.RA_ERR_INVALID_ARG),      # output overlaps q8
+    (dict(lse=SV), _lib.RA_ERR_INVALID_ARG),            # lse overlaps sv
+    (dict(lse=O + 64), _lib.RA_ERR_INVALID_ARG),        # lse overlaps out
+])
+def test_fwd_fp8_rejects_invalid_arguments(lib, kw, status):
+    assert fp8_status(lib, **kw) == status
+    assert _lib.last_error()
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(L=0), dict(Hq=0, Hkv=0)])
+def test_fwd_fp8_empty_problem_launches_nothing(lib, kw):
+    assert fp8_status(lib, q8=0, k8=0, v8=0, sq=0, sk=0, sv=0, out=0, lse=0, **kw) == _lib.RA_OK
+
+
+def quant_status(lib, **kw):
+    args = dict(x=Q, codes=K, scales=SQ, B=1, L=300, H=2, d=128)
+    args.update(kw)
+    return lib.ring_attn_quantize_fp8(args["x"], args["codes"], args["scales"], args["B"],
+                                      args["L"], args["H"], args["d"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=12), _lib.RA_ERR_UNSUPPORTED),
+    (dict(d=0), _lib.RA_ERR_UNSUPPORTED),
+    (dict(d=264), _lib.RA_ERR_UNSUPPORTED),
+    (dict(H=70000), _lib.RA_ERR_UNSUPPORTED),
+    (dict(B=-1), _lib.RA_ERR_INVALID_ARG),
+    (dict(x=0), _lib.RA_ERR_INVALID_ARG),
+    (dict(codes=K + 8), _lib.RA_ERR_INVALID_ARG),       # not 16-byte aligned
+    (dict(scales=SQ + 2), _lib.RA_ERR_INVALID_ARG),     # not 4-byte aligned
+    (dict(codes=Q + 64), _lib.RA_ERR_INVALID_ARG),      # codes overlap x
+    (dict(scales=K + 16), _lib.RA_ERR_INVALID_ARG),     # scales overlap codes
+])
+def test_quantize_fp8_rejects_invalid_arguments(lib, kw, status):
+    assert quant_status(lib, **kw) == status
+    assert _lib.last_error()
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(L=0), dict(H=0)])
+def test_quantize_fp8_empty_launches_nothing(lib, kw):
+    assert quant_status(lib, x=0, codes=0, scales=0, **kw) == _lib.RA_OK
