@@ -118,17 +118,26 @@ KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd.cu",
 TRAFFIC_RECORD = "profiles/ra_fwd_l128k_h32_causal_dram.md"
 
 
-def recorded_traffic(workload_name: str):
-    """DRAM bytes per launch from the committed ncu record, or None when the
+FP8_KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd_fp8.cu",
+                      "ring_attention_ordered_b200/csrc/ptx_sm100.cuh",
+                      "ring_attention_ordered_b200/csrc/ra_api.cu",
+                      "ring_attention_ordered_b200/csrc/ra_internal.h",
+                      "ring_attention_ordered_b200/csrc/ra_sync.cuh",
+                      "ring_attention_ordered_b200/csrc/ra_schedule.cuh"]
+FP8_TRAFFIC_RECORD = "profiles/ra_fwd_fp8_l128k_h32_causal_dram.md"
+
+
+def recorded_traffic(workload_name: str, record: str = TRAFFIC_RECORD, sources=None):
+    """DRAM bytes per launch from a committed ncu record, or None when the
     workload differs or the kernel sources changed since the capture."""
     import hashlib
     import re
     if workload_name != "l128k_h32_causal":
         return None
     try:
-        text = open(os.path.join(ROOT, TRAFFIC_RECORD)).read()
+        text = open(os.path.join(ROOT, record)).read()
         h = hashlib.sha256()
-        for f in KERNEL_SOURCES:
+        for f in (KERNEL_SOURCES if sources is None else sources):
             with open(os.path.join(ROOT, f), "rb") as fh:
                 h.update(fh.read())
     except OSError:
@@ -270,7 +279,9 @@ def time_fp8(api, q, k, v, w, stream, steps: int, peaks: dict, world: int = 1, d
     return {
         "ms": ms, "TFLOP/s": world * achieved, "steps": steps, "launches_per_call": 1,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                     "frac": achieved / peak, "traffic": None, "kernel": "ra_fwd_fp8_kernel",
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(w.name, FP8_TRAFFIC_RECORD, FP8_KERNEL_SOURCES),
+                     "kernel": "ra_fwd_fp8_kernel",
                      "peak_kind": "E4M3 dense = 2 x bf16_tflops_sustained "
                                   f"({peaks['source']}), the nominal 4.5 / 2.25 PFLOP/s ratio"},
         "frac_of_bf16_sustained": achieved / peaks["bf16_tflops_sustained"],
