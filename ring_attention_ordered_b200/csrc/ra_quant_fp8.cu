@@ -8,10 +8,10 @@
 // E4M3 with ties to even, saturating at +-448.  A ragged last tile holds the
 // remaining rows.
 //
-// One CTA per (tile, head, batch): 256 threads load the tile's rows (d bf16
-// values each, 16 bytes per load) into registers once, reduce |x| to the
-// tile's maximum, and write the codes (8 bytes per store) and the scale.  The
-// kernel is bound by HBM: 2 bytes read and 1 byte written per element.
+// One CTA per (tile, head, batch), 256 threads: a first pass of 16-byte loads
+// reduces |x| to the tile's maximum, a second pass reads the tile again (an
+// L2 hit) and writes the codes (8 bytes per store) and the scale.  The kernel
+// is bound by HBM: 2 bytes read and 1 byte written per element.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -55,15 +55,14 @@ __global__ void __launch_bounds__(QT) ra_quant_fp8_kernel(const __nv_bfloat16* _
   const long long row_stride = static_cast<long long>(H) * d;
   const long long base = (static_cast<long long>(b) * L + r0) * row_stride + static_cast<long long>(h) * d;
 
-  uint4 v[MAX_CHUNKS];
+  // pass 1: the tile's maximum magnitude (loads only, all in flight at once)
   float m = 0.f;
 #pragma unroll
   for (int i = 0; i < MAX_CHUNKS; ++i) {
     const int c = threadIdx.x + i * QT;
     if (c < n) {
       const int r = c / cpr, cc = c % cpr;
-      v[i] = __ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc);
-      m = absmax8(v[i], m);
+      m = absmax8(__ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc), m);
     }
   }
 #pragma unroll
@@ -76,12 +75,16 @@ __global__ void __launch_bounds__(QT) ra_quant_fp8_kernel(const __nv_bfloat16* _
   const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
   if (threadIdx.x == 0) scales[(static_cast<long long>(b) * H + h) * T + t] = s;
 
-#pragma unroll
+  // pass 2: read the tile again (from L2: it was read a moment ago) and
+  // write the codes.  Holding the tile in registers between the passes
+  // instead would cut the resident CTAs per SM from 8 to 3.
+#pragma unroll 4
   for (int i = 0; i < MAX_CHUNKS; ++i) {
     const int c = threadIdx.x + i * QT;
     if (c < n) {
       const int r = c / cpr, cc = c % cpr;
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc);
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
       uint32_t w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
