@@ -25,6 +25,14 @@ def _check_cuda(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
 
 
+def _check_out(t: torch.Tensor, name: str, dtype: torch.dtype, shape):
+    """A caller-supplied output must match the shape the kernel writes: the
+    library writes through raw pointers and cannot see a buffer's size."""
+    _check_cuda(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: bool,
         scale: float | None = None, out: torch.Tensor | None = None,
         lse: torch.Tensor | None = None, stream=None):
@@ -43,8 +51,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
-    _check_cuda(out, "out", torch.bfloat16, 4)
-    _check_cuda(lse, "lse", torch.float32, 3)
+    _check_out(out, "out", torch.bfloat16, (B, L, Hq, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq, L))
     with torch.cuda.device(q.device):
         _lib.ring_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                            lse.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale,
@@ -106,6 +114,11 @@ def bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
     _check_cuda(lse, "lse", torch.float32, 3)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
+    if k.shape != (B, L, Hkv, d) or v.shape != k.shape or out.shape != q.shape or \
+            dout.shape != q.shape or lse.shape != (B, Hq, L):
+        raise ValueError("k/v/out/dout/lse shapes do not match q")
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _check_out(t, n, torch.bfloat16, tuple(ref.shape))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     with torch.cuda.device(q.device):
@@ -155,7 +168,9 @@ def round_bf16(src: torch.Tensor, dst: torch.Tensor | None = None, stream=None):
     """fp32 -> bf16 (nearest even) through ring_attn_round_bf16."""
     if not src.is_cuda or src.dtype != torch.float32 or not src.is_contiguous():
         raise TypeError("src must be a contiguous fp32 CUDA tensor")
-    dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device) if dst is None else dst
+    if dst is None:
+        dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    _check_out(dst, "dst", torch.bfloat16, tuple(src.shape))
     with torch.cuda.device(src.device):
         _lib.ring_attn_round_bf16(src.data_ptr(), dst.data_ptr(), src.numel(),
                                   _stream_handle(stream))
@@ -206,8 +221,8 @@ def quantize_fp8(x: torch.Tensor, codes: torch.Tensor | None = None,
         codes = torch.empty((B, L, H, d), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((B, H, (L + 127) // 128), dtype=torch.float32, device=x.device)
-    _check_cuda(codes, "codes", torch.uint8, 4)
-    _check_cuda(scales, "scales", torch.float32, 3)
+    _check_out(codes, "codes", torch.uint8, (B, L, H, d))
+    _check_out(scales, "scales", torch.float32, (B, H, (L + 127) // 128))
     with torch.cuda.device(x.device):
         _lib.ring_attn_quantize_fp8(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), B, L, H, d,
                                     _stream_handle(stream))
@@ -240,8 +255,8 @@ def fwd_fp8(q8: torch.Tensor, sq: torch.Tensor, k8: torch.Tensor, sk: torch.Tens
         out = torch.empty((B, L, Hq, d), dtype=torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q8.device)
-    _check_cuda(out, "out", torch.bfloat16, 4)
-    _check_cuda(lse, "lse", torch.float32, 3)
+    _check_out(out, "out", torch.bfloat16, (B, L, Hq, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq, L))
     with torch.cuda.device(q8.device):
         _lib.ring_attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), sq.data_ptr(),
                                sk.data_ptr(), sv.data_ptr(), out.data_ptr(), lse.data_ptr(), B,
@@ -257,10 +272,14 @@ def merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torc
     _check_cuda(lse_a, "lse_a", torch.float32, 1)
     _check_cuda(lse_b, "lse_b", torch.float32, 1)
     rows, d = o_a.shape
+    if tuple(o_b.shape) != (rows, d) or tuple(lse_a.shape) != (rows,) or tuple(lse_b.shape) != (rows,):
+        raise ValueError("o_a, o_b must be [rows, d] and lse_a, lse_b [rows]")
     if out is None:
         out = torch.empty_like(o_a)
     if lse_out is None:
         lse_out = torch.empty_like(lse_a)
+    _check_out(out, "out", torch.float32, (rows, d))
+    _check_out(lse_out, "lse_out", torch.float32, (rows,))
     with torch.cuda.device(o_a.device):
         _lib.ring_attn_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
                              out.data_ptr(), lse_out.data_ptr(), rows, d, _stream_handle(stream))
