@@ -346,7 +346,8 @@ ra_status ring_attn_set_wait_limit_ns(uint64_t ns);
  * SM, the default).  Process-wide; used to exercise the scheduler. */
 ra_status ring_attn_set_max_ctas(int n);
 
-/* Order in which the forward kernel's persistent CTAs take work units (a unit
+/* Order in which the forward kernels' persistent CTAs (bf16 and FP8) take
+ * work units (a unit
  * = two 128-row query tiles sharing one K/V stream; causal units differ in
  * length).  Results do not depend on it.  Process-wide.
  *   RA_SCHEDULE_AUTO (default): HEAD_MAJOR when the K/V tensors exceed
