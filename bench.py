@@ -645,6 +645,31 @@ def run_bwd_only(args, w):
     return 0
 
 
+def run_fp8_only(args, w):
+    """Only the FP8 leg on one GPU: block quantisation of the workload's q, k,
+    v, then W = 2 warm-up and K timed ring_attn_fwd_fp8 launches; one JSON
+    line (a small command for profiling the FP8 kernel alone)."""
+    import torch
+
+    from ring_attention_ordered_b200 import _lib, api
+    from ring_attention_ordered_b200.inputs import workload_inputs
+
+    if not fp8_supported(w):
+        print(json.dumps({"kind": "fp8", "name": w.name,
+                          "unavailable": "the FP8 forward needs d = 128 and L / n_ring a "
+                                         "multiple of 128"}), flush=True)
+        return 0
+    _lib.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    q, k, v = (t.to(dev) for t in workload_inputs(w))
+    stream = torch.cuda.current_stream(dev)
+    f8 = time_fp8(api, q, k, v, w, stream, args.steps, peaks)
+    print(json.dumps({"kind": "fp8", "workload": w.describe(), "name": w.name, **f8}), flush=True)
+    return 0
+
+
 def run_ring_emulated(args, w):
     """The multi-host ring's compute, host by host, on one GPU (not the
     contract line).  For each layout, every host's visit sequence on the
@@ -765,6 +790,8 @@ def main():
                     help="print one line per named workload instead of the benchmark line")
     ap.add_argument("--bwd-only", action="store_true",
                     help="time only the backward pass on the workload")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="time only the FP8 forward (and its quantiser) on the workload")
     ap.add_argument("--ring-emulated", action="store_true",
                     help="time every host of the multi-host ring on this GPU (three layouts)")
     ap.add_argument("--ref-budget", type=float, default=None,
@@ -783,6 +810,8 @@ def main():
         return run_ring_emulated(args, w)
     if args.bwd_only:
         return run_bwd_only(args, w)
+    if args.fp8_only:
+        return run_fp8_only(args, w)
     return run_ours(args, w, world, rank, local)
 
 
