@@ -246,6 +246,9 @@ def fwd_fp8(q8: torch.Tensor, sq: torch.Tensor, k8: torch.Tensor, sk: torch.Tens
     if k8.shape != (B, L, Hkv, d) or v8.shape != k8.shape:
         raise ValueError(f"k8/v8 shape {tuple(k8.shape)}/{tuple(v8.shape)} does not match "
                          f"q8 {tuple(q8.shape)}")
+    if L % 128 != 0 or (n_ring > 0 and (L // n_ring) % 128 != 0):
+        raise ValueError(f"the FP8 forward needs L / n_ring to be a multiple of 128 "
+                         f"(L={L}, n_ring={n_ring})")
     T = L // 128
     if sq.shape != (B, Hq, T) or sk.shape != (B, Hkv, T) or sv.shape != (B, Hkv, T):
         raise ValueError("scale tensors must be [B, H, L/128]")
