@@ -1,4 +1,4 @@
-"""Fit the polynomial the forward kernel uses for part of its 2^x evaluations.
+"""Fit the polynomial the kernels can use for part of their 2^x evaluations.
 
 Method: Remez exchange (minimax in relative error) for p(f) ~ 2^f on
 f in [-1/2, 1/2], degree 3.  The kernel splits x = j + f with j = round(x)
@@ -9,7 +9,8 @@ Horner evaluation.
 
 Run: ``python ring_attention_ordered_b200/csrc/fit_exp2_poly.py`` -- prints
 the coefficients (c0 + c1 f + c2 f^2 + c3 f^3) and the maximum relative
-error; the values are copied into ``ra_fwd.cu`` (EXP2_C0..C3).
+error; the values are copied into ``ra_exp2.cuh`` (EXP2_C0..C3), which
+``tests/test_exp2_poly.py`` checks against this fit.
 """
 
 from __future__ import annotations
