@@ -42,7 +42,7 @@ typedef struct CUstream_st* ra_stream_t;
 typedef enum {
   RA_OK = 0,
   RA_ERR_INVALID_ARG = 1,  /* a shape, pointer, alignment or value is invalid   */
-  RA_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements  */
+  RA_ERR_UNSUPPORTED = 2,  /* valid request outside what this library implements */
   RA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                 */
   RA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (see below)    */
 } ra_status;
