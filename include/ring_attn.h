@@ -25,6 +25,10 @@
  *     device variables of the module: three status words per device (bf16
  *     forward, backward and FP8 forward kernels) and the fixed 4 MiB array
  *     of ring_attn_bwd_noalloc.
+ *   - Contexts: a call runs in the calling thread's current CUDA context,
+ *     the device's primary context or one the caller created (cuCtxCreate),
+ *     and `stream` must belong to that context.  A thread with no current
+ *     context gets the primary context of its current device made current.
  */
 #ifndef RING_ATTN_H_
 #define RING_ATTN_H_
@@ -245,9 +249,12 @@ ra_status ring_attn_round_bf16(const float* src, void* dst, int64_t n, ra_stream
  * two calls whose kernels may run at the same time (on different streams,
  * or from different host threads) race on it and corrupt each other's
  * results: order them on one stream, or use ring_attn_bwd with a workspace
- * per concurrent call.  The first call on each device looks up the array's
- * address (cudaGetSymbolAddress) and caches it; make that first call before
- * any stream capture begins.
+ * per concurrent call.  The array belongs to the module loaded in each CUDA
+ * context.  A call made while `stream` is not capturing looks up the array's
+ * address in the current context (cudaGetSymbolAddress) and remembers it for
+ * that context.  A call made during a stream capture uses the remembered
+ * address, so make the first call in each context before any stream capture
+ * begins.
  */
 ra_status ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,

@@ -1,10 +1,19 @@
 """Torch-facing wrapper: checks tensors, allocates outputs with torch and
-passes raw pointers plus the current CUDA stream to the C ABI.  All
-arithmetic happens in the library's kernels."""
+passes raw pointers plus a CUDA stream (the caller's ``stream``, else the
+current one) to the C ABI.  All arithmetic happens in the library's kernels.
+
+Outputs and temporaries that a call allocates are allocated while the stream
+the kernels run on is current.  torch's caching allocator ties a block to the
+stream that was current at allocation and reuses it only in that stream's
+order.  A temporary freed when the call returns, such as the backward's
+workspace, is therefore not handed to other work before the kernels that use
+it have finished.
+"""
 
 from __future__ import annotations
 
 import math
+from contextlib import contextmanager
 
 import torch
 
@@ -14,6 +23,16 @@ from . import _lib
 def _stream_handle(stream) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(s.cuda_stream)
+
+
+@contextmanager
+def _on(device, stream):
+    """Make ``device`` and the call's stream current; yields the stream
+    handle for the C ABI."""
+    with torch.cuda.device(device):
+        s = stream if stream is not None else torch.cuda.current_stream(device)
+        with torch.cuda.stream(s):
+            yield int(s.cuda_stream)
 
 
 def _check_cuda(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
@@ -47,16 +66,15 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ring: int, causal: 
         raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
-    _check_out(out, "out", torch.bfloat16, (B, L, Hq, d))
-    _check_out(lse, "lse", torch.float32, (B, Hq, L))
-    with torch.cuda.device(q.device):
+    with _on(q.device, stream) as sh:
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+        _check_out(out, "out", torch.bfloat16, (B, L, Hq, d))
+        _check_out(lse, "lse", torch.float32, (B, Hq, L))
         _lib.ring_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                           lse.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale,
-                           _stream_handle(stream))
+                           lse.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale, sh)
     return out, lse
 
 
@@ -80,24 +98,24 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
         raise ValueError("out/dout/lse shapes do not match q")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
-        _check_cuda(t, n, torch.bfloat16, 4)
-        if t.shape != ref.shape:
-            raise ValueError(f"{n} shape does not match")
-    need = _lib.ring_attn_bwd_workspace_size(B, Hq, L)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if not workspace.is_cuda or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor")
-    ws_bytes = workspace.numel() * workspace.element_size()
-    with torch.cuda.device(q.device):
+    with _on(q.device, stream) as sh:
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+            _check_cuda(t, n, torch.bfloat16, 4)
+            if t.shape != ref.shape:
+                raise ValueError(f"{n} shape does not match")
+        need = _lib.ring_attn_bwd_workspace_size(B, Hq, L)
+        if workspace is None:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_bytes = workspace.numel() * workspace.element_size()
         _lib.ring_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                            dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                            dv.data_ptr(), workspace.data_ptr(), ws_bytes, B, Hq, Hkv, L, d,
-                           n_ring, causal, scale, _stream_handle(stream))
+                           n_ring, causal, scale, sh)
     return dq, dk, dv
 
 
@@ -121,11 +139,10 @@ def bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
         _check_out(t, n, torch.bfloat16, tuple(ref.shape))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    with torch.cuda.device(q.device):
+    with _on(q.device, stream) as sh:
         _lib.ring_attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                    dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                   dv.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale,
-                                   _stream_handle(stream))
+                                   dv.data_ptr(), B, Hq, Hkv, L, d, n_ring, causal, scale, sh)
     return dq, dk, dv
 
 
@@ -156,24 +173,23 @@ def bwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tens
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     ptr = lambda t: 0 if t is None else t.data_ptr()  # noqa: E731
-    with torch.cuda.device(q.device):
+    with _on(q.device, stream) as sh:
         _lib.ring_attn_bwd_visit(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                  dout.data_ptr(), lse.data_ptr(), ptr(dq_acc), ptr(dk_acc),
                                  ptr(dv_acc), ptr(dq), workspace.data_ptr(),
                                  workspace.numel() * workspace.element_size(), B, Hq, Hkv, l, d,
-                                 diag, parts, fold_q, fold_kv, scale, _stream_handle(stream))
+                                 diag, parts, fold_q, fold_kv, scale, sh)
 
 
 def round_bf16(src: torch.Tensor, dst: torch.Tensor | None = None, stream=None):
     """fp32 -> bf16 (nearest even) through ring_attn_round_bf16."""
     if not src.is_cuda or src.dtype != torch.float32 or not src.is_contiguous():
         raise TypeError("src must be a contiguous fp32 CUDA tensor")
-    if dst is None:
-        dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
-    _check_out(dst, "dst", torch.bfloat16, tuple(src.shape))
-    with torch.cuda.device(src.device):
-        _lib.ring_attn_round_bf16(src.data_ptr(), dst.data_ptr(), src.numel(),
-                                  _stream_handle(stream))
+    with _on(src.device, stream) as sh:
+        if dst is None:
+            dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+        _check_out(dst, "dst", torch.bfloat16, tuple(src.shape))
+        _lib.ring_attn_round_bf16(src.data_ptr(), dst.data_ptr(), src.numel(), sh)
     return dst
 
 
@@ -202,10 +218,10 @@ def fwd_visit(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Te
             raise ValueError("out shape does not match q")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    with torch.cuda.device(q.device):
+    with _on(q.device, stream) as sh:
         _lib.ring_attn_fwd_visit(q.data_ptr(), k.data_ptr(), v.data_ptr(), o_acc.data_ptr(),
                                  lse_acc.data_ptr(), 0 if out is None else out.data_ptr(),
-                                 B, Hq, Hkv, l, d, diag, fold, scale, _stream_handle(stream))
+                                 B, Hq, Hkv, l, d, diag, fold, scale, sh)
     return o_acc, lse_acc, out
 
 
@@ -217,15 +233,15 @@ def quantize_fp8(x: torch.Tensor, codes: torch.Tensor | None = None,
     (``codes.view(torch.float8_e4m3fn)`` reads them as FP8)."""
     _check_cuda(x, "x", torch.bfloat16, 4)
     B, L, H, d = x.shape
-    if codes is None:
-        codes = torch.empty((B, L, H, d), dtype=torch.uint8, device=x.device)
-    if scales is None:
-        scales = torch.empty((B, H, (L + 127) // 128), dtype=torch.float32, device=x.device)
-    _check_out(codes, "codes", torch.uint8, (B, L, H, d))
-    _check_out(scales, "scales", torch.float32, (B, H, (L + 127) // 128))
-    with torch.cuda.device(x.device):
+    with _on(x.device, stream) as sh:
+        if codes is None:
+            codes = torch.empty((B, L, H, d), dtype=torch.uint8, device=x.device)
+        if scales is None:
+            scales = torch.empty((B, H, (L + 127) // 128), dtype=torch.float32, device=x.device)
+        _check_out(codes, "codes", torch.uint8, (B, L, H, d))
+        _check_out(scales, "scales", torch.float32, (B, H, (L + 127) // 128))
         _lib.ring_attn_quantize_fp8(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), B, L, H, d,
-                                    _stream_handle(stream))
+                                    sh)
     return codes, scales
 
 
@@ -254,16 +270,16 @@ def fwd_fp8(q8: torch.Tensor, sq: torch.Tensor, k8: torch.Tensor, sk: torch.Tens
         raise ValueError("scale tensors must be [B, H, L/128]")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if out is None:
-        out = torch.empty((B, L, Hq, d), dtype=torch.bfloat16, device=q8.device)
-    if lse is None:
-        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q8.device)
-    _check_out(out, "out", torch.bfloat16, (B, L, Hq, d))
-    _check_out(lse, "lse", torch.float32, (B, Hq, L))
-    with torch.cuda.device(q8.device):
+    with _on(q8.device, stream) as sh:
+        if out is None:
+            out = torch.empty((B, L, Hq, d), dtype=torch.bfloat16, device=q8.device)
+        if lse is None:
+            lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q8.device)
+        _check_out(out, "out", torch.bfloat16, (B, L, Hq, d))
+        _check_out(lse, "lse", torch.float32, (B, Hq, L))
         _lib.ring_attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), sq.data_ptr(),
                                sk.data_ptr(), sv.data_ptr(), out.data_ptr(), lse.data_ptr(), B,
-                               Hq, Hkv, L, d, n_ring, causal, scale, _stream_handle(stream))
+                               Hq, Hkv, L, d, n_ring, causal, scale, sh)
     return out, lse
 
 
@@ -277,15 +293,15 @@ def merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torc
     rows, d = o_a.shape
     if tuple(o_b.shape) != (rows, d) or tuple(lse_a.shape) != (rows,) or tuple(lse_b.shape) != (rows,):
         raise ValueError("o_a, o_b must be [rows, d] and lse_a, lse_b [rows]")
-    if out is None:
-        out = torch.empty_like(o_a)
-    if lse_out is None:
-        lse_out = torch.empty_like(lse_a)
-    _check_out(out, "out", torch.float32, (rows, d))
-    _check_out(lse_out, "lse_out", torch.float32, (rows,))
-    with torch.cuda.device(o_a.device):
+    with _on(o_a.device, stream) as sh:
+        if out is None:
+            out = torch.empty_like(o_a)
+        if lse_out is None:
+            lse_out = torch.empty_like(lse_a)
+        _check_out(out, "out", torch.float32, (rows, d))
+        _check_out(lse_out, "lse_out", torch.float32, (rows,))
         _lib.ring_attn_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
-                             out.data_ptr(), lse_out.data_ptr(), rows, d, _stream_handle(stream))
+                             out.data_ptr(), lse_out.data_ptr(), rows, d, sh)
     return out, lse_out
 
 

@@ -51,6 +51,31 @@ ra_status ok() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
+namespace ra {
+
+// The calling thread's current driver context (nullptr if none), through the
+// driver entry point the runtime exposes (no link against libcuda).
+cudaError_t current_context(CUcontext* ctx) {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  if (!fn) return cudaErrorNotSupported;
+  *ctx = nullptr;
+  return fn(ctx) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+
+}  // namespace ra
+
+namespace {
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -65,16 +90,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// Query SM count and compute capability of the current device once.  Also
-// makes the device's primary context current on the calling thread: a thread
-// that has only been told its device (such as torch's autograd worker) may
-// have none yet, and the tensor-map encoder needs one.
+// Query SM count and compute capability of the current device once.  A
+// thread with no current context (one that has only been told its device,
+// such as torch's autograd worker) gets the device's primary context made
+// current, since the tensor-map encoder needs a context; a context the caller
+// made current itself (primary or its own, cuCtxCreate) is left in place and
+// used.
 ra_status device_info(int* sms) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(RA_ERR_UNSUPPORTED, "device index %d", dev);
-  if ((e = cudaSetDevice(dev)) != cudaSuccess)
+  CUcontext cur = nullptr;
+  if ((e = ra::current_context(&cur)) != cudaSuccess)
+    return fail(RA_ERR_CUDA, "cuCtxGetCurrent: %s", cudaGetErrorString(e));
+  if (cur == nullptr && (e = cudaSetDevice(dev)) != cudaSuccess)
     return fail(RA_ERR_CUDA, "cudaSetDevice: %s", cudaGetErrorString(e));
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_cc_ok[dev] == 0) {
@@ -457,7 +487,7 @@ ra_status ring_attn_bwd_noalloc(const void* q, const void* k, const void* v, con
     return ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, nullptr, 0, B, Hq, Hkv, L, d,
                          n_ring, causal, scale, stream);
   void* scratch = nullptr;
-  cudaError_t e = ra::noalloc_scratch(&scratch);
+  cudaError_t e = ra::noalloc_scratch(&scratch, stream);
   if (e != cudaSuccess)
     return fail(RA_ERR_CUDA, "static scratch lookup: %s", cudaGetErrorString(e));
   return ring_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, scratch,

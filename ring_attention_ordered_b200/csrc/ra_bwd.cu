@@ -43,7 +43,6 @@
 #include <mutex>
 
 #include "ptx_sm100.cuh"
-#include "ra_exp2.cuh"
 #include "ra_internal.h"
 #include "ra_sync.cuh"
 #include "ring_attn.h"
@@ -63,14 +62,6 @@ constexpr int WARP_LOAD = 8;
 constexpr int WARP_MMA = 9;
 constexpr int HALF = 64;             // columns per softmax warpgroup
 constexpr float LOG2E = 1.4426950408889634f;
-// Column pairs j (of a warpgroup's 32) with j % EMU == EMU - 1 take 2^x from
-// the polynomial on the FMA pipe, the others from MUFU ex2 (0, the default:
-// all from MUFU; one pair in 4, 3 or 2 on the polynomial measured 1-4%
-// slower on B200).
-#ifndef RA_BWD_EMU_PERIOD
-#define RA_BWD_EMU_PERIOD 0
-#endif
-constexpr int EMU = RA_BWD_EMU_PERIOD;
 
 
 // Device status word of the backward kernels: 0 = ok, else (code << 32) | where.
@@ -525,14 +516,9 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, i
         const uint64_t x2 =
             f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])), c2x2, nl2);
         float p0, p1;
-        if (EMU > 0 && (j % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-          exp2_poly2(x2, p0, p1);
-        } else {
-          float e0, e1;
-          f2_unpack(x2, e0, e1);
-          p0 = ex2_approx(e0);
-          p1 = ex2_approx(e1);
-        }
+        f2_unpack(x2, p0, p1);
+        p0 = ex2_approx(p0);
+        p1 = ex2_approx(p1);
         if (masked) {
           p0 = (2 * j > lim_local) ? 0.f : p0;
           p1 = (2 * j + 1 > lim_local) ? 0.f : p1;
@@ -968,14 +954,9 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
         const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])),
                                    c2x2, f2_pack(l2.x, l2.y));
         float p0, p1;
-        if (EMU > 0 && (j % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-          exp2_poly2(x2, p0, p1);
-        } else {
-          float e0, e1;
-          f2_unpack(x2, e0, e1);
-          p0 = ex2_approx(e0);
-          p1 = ex2_approx(e1);
-        }
+        f2_unpack(x2, p0, p1);
+        p0 = ex2_approx(p0);
+        p1 = ex2_approx(p1);
         if (diag) {
           p0 = (2 * j < first) ? 0.f : p0;
           p1 = (2 * j + 1 < first) ? 0.f : p1;
@@ -1146,19 +1127,36 @@ cudaError_t launch_bwd(const BwdParams& prm, int d, int num_sms, int max_ctas,
 // overwrites the entries it reads, so nothing in it has to start at zero.
 __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchRows];
 
-cudaError_t noalloc_scratch(void** ptr) {
+cudaError_t noalloc_scratch(void** ptr, cudaStream_t stream) {
+  struct Entry {
+    CUcontext ctx;
+    void* addr;
+  };
   static std::mutex mu;
-  static void* addr[64] = {nullptr};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static Entry cache[64] = {};
+  static int n_cached = 0;
+  CUcontext ctx = nullptr;
+  cudaError_t e = current_context(&ctx);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    e = cudaGetSymbolAddress(&addr[dev], g_noalloc_scratch);
+  int slot = -1;
+  for (int i = 0; i < n_cached; ++i)
+    if (cache[i].ctx == ctx) slot = i;
+  if (cs == cudaStreamCaptureStatusNone || slot < 0 || ctx == nullptr) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
+    // the lookup made a context current if there was none
+    if (ctx == nullptr && (e = current_context(&ctx)) != cudaSuccess) return e;
+    for (int i = 0; i < n_cached; ++i)
+      if (cache[i].ctx == ctx) slot = i;
+    if (slot < 0) slot = (n_cached < 64) ? n_cached++ : 0;
+    cache[slot] = Entry{ctx, addr};
   }
-  *ptr = addr[dev];
+  *ptr = cache[slot].addr;
   return cudaSuccess;
 }
 

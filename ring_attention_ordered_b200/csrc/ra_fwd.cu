@@ -41,7 +41,6 @@
 
 #include "ptx_sm100.cuh"
 #include "ra_internal.h"
-#include "ra_exp2.cuh"
 #include "ra_merge_math.cuh"
 #include "ra_schedule.cuh"
 #include "ra_sync.cuh"
@@ -66,18 +65,6 @@ constexpr int CONTROL_REGS = 56;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
 constexpr float RESCALE_LOG2 = 8.0f;
-// Columns (out of 128) of each score row whose 2^x is evaluated with a
-// polynomial on the FMA pipe instead of the MUFU ex2 unit: at full tensor rate
-// one MUFU ex2 per score element would keep MUFU exactly as busy as the
-// tensor core, so part of the exponentials move to the otherwise idle FMA
-// pipe.
-// Column pairs j (0..63) with (j % EMU_PERIOD) == EMU_PERIOD - 1 use the
-// polynomial; 0 disables it.  Spreading them across the row lets the
-// scheduler overlap them with the MUFU work of the other pairs.
-#ifndef RA_EMU_PERIOD
-#define RA_EMU_PERIOD 0
-#endif
-constexpr int EMU_PERIOD = RA_EMU_PERIOD;
 constexpr float LN2 = 0.69314718055994530942f;
 
 // Device status word: 0 = ok, otherwise (code << 32) | where.
@@ -375,19 +362,23 @@ drain:
 
 // ------------------------------------------------------------------ softmax
 // One score row (128 columns held in sr): P = 2^(s * c2 - m) written as bf16
-// pairs to TMEM columns [0, 64) at tS, returns the row sum of the fp32 P.
-// Arrives on p_half_bar once the first 64 keys of P are stored.
+// pairs to TMEM columns [0, 64) at tS.  Returns the row sums of the fp32 P
+// (x, for the log-sum-exp) and of the bf16-rounded P that the P V product
+// uses (y, which normalises O, so that O is exactly the weighted mean of the
+// V rows under the rounded weights).  Arrives on p_half_bar once the first
+// 64 keys of P are stored.
 // MASKED: columns > lim are excluded (set to zero exactly).  Issues
 // warp-collective tcgen05.st: every lane of the warp must call the same
 // instantiation at the same time.
 template <bool MASKED>
-__device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, float m, int lim,
-                                               uint32_t tS, uint32_t p_half_bar) {
+__device__ __forceinline__ float2 exp_row_store(uint32_t (&sr)[128], float c2, float m, int lim,
+                                                uint32_t tS, uint32_t p_half_bar) {
   const uint64_t c2x2 = f2_pack(c2, c2);
   const uint64_t nm2 = f2_pack(-m, -m);
-  uint64_t acc[4];
+  uint64_t acc[4], accr[2];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
+  accr[0] = accr[1] = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     uint32_t pk[32];
@@ -397,20 +388,17 @@ __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, fl
       const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])),
                                  c2x2, nm2);
       float p0, p1;
-      if (EMU_PERIOD > 0 && (j % (EMU_PERIOD > 0 ? EMU_PERIOD : 1)) == EMU_PERIOD - 1) {
-        exp2_poly2(x2, p0, p1);
-      } else {
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        p0 = ex2_approx(x0);
-        p1 = ex2_approx(x1);
-      }
+      f2_unpack(x2, p0, p1);
+      p0 = ex2_approx(p0);
+      p1 = ex2_approx(p1);
       if (MASKED) {
         p0 = (col > lim) ? 0.f : p0;
         p1 = (col + 1 > lim) ? 0.f : p1;
       }
       acc[j & 3] = f2_add(acc[j & 3], f2_pack(p0, p1));
       pk[j] = pack_bf16x2(p0, p1);
+      accr[j & 1] = f2_add(accr[j & 1], f2_pack(__uint_as_float(pk[j] << 16),
+                                                __uint_as_float(pk[j] & 0xffff0000u)));
     }
     tmem_st32(tS + 32 * half, pk);
     if (half == 0) {
@@ -422,9 +410,10 @@ __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, fl
   }
   const uint64_t s01 = f2_add(acc[0], acc[1]);
   const uint64_t s23 = f2_add(acc[2], acc[3]);
-  float a, b;
+  float a, b, ar, br;
   f2_unpack(f2_add(s01, s23), a, b);
-  return a + b;
+  f2_unpack(f2_add(accr[0], accr[1]), ar, br);
+  return make_float2(a + b, ar + br);
 }
 
 // Epilogue of a per-visit launch: this visit's normalised rows O / l (fp32)
@@ -496,7 +485,9 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
     const int qt = w ? x.qt[1] : x.qt[0];
     const int h = w ? x.h[1] : x.h[0];
     const int qrow = qt * BM + t;                  // row inside the ring block
-    float m = -INFINITY, l = 0.f;
+    // running max m (log2 units); row sums of the unrounded P (l, for the
+    // lse) and of the bf16-rounded P (lr, for O)
+    float m = -INFINITY, l = 0.f, lr = 0.f;
     KvIter it;
     it.start(p, x);
 
@@ -575,9 +566,10 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
         }
         m = m_new;
       }
-      const float rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS, br.p_half(w))
-                                : exp_row_store<false>(sr, c2, m, lim, tS, br.p_half(w));
-      l = l * alpha + rsum;
+      const float2 rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS, br.p_half(w))
+                                 : exp_row_store<false>(sr, c2, m, lim, tS, br.p_half(w));
+      l = l * alpha + rsum.x;
+      lr = lr * alpha + rsum.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(br.p_full(w));
@@ -590,11 +582,11 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
       tc_fence_after();
       const bool row_ok = qrow < p.blk_len;
       const long long pos = static_cast<long long>(x.blk) * p.blk_len + qrow;
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / lr;
       if (p.o_acc != nullptr) {
         // a row with no allowed key (strict diagonal, row 0) is an empty
         // partial: o = 0, lse = -inf, which the fold ignores
-        visit_epilogue<D>(p, tO, row_ok, x.b, pos, h, l > 0.f ? inv_l : 0.f, (m + log2f(l)) * LN2);
+        visit_epilogue<D>(p, tO, row_ok, x.b, pos, h, lr > 0.f ? inv_l : 0.f, (m + log2f(l)) * LN2);
         tc_fence_before();
         mbar_arrive(br.o_free(w));
         ++units_w;

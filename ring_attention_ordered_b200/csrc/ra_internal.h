@@ -115,8 +115,14 @@ cudaError_t read_and_clear_bwd_status(unsigned long long* out);
 
 // Static scratch of ring_attn_bwd_noalloc (fp32 entries, 4 MiB).
 constexpr long long kNoAllocScratchRows = 1ll << 20;
-// Address of that scratch on the current device (looked up once per device).
-cudaError_t noalloc_scratch(void** ptr);
+// Device address of that scratch in the current context.  Looked up on every
+// call made while `stream` is not capturing (the module, and so the address,
+// belongs to a context, which cudaDeviceReset or a caller's own context can
+// change); during a capture the address cached for the current context is
+// used, so a context's first call must come before any capture.
+cudaError_t noalloc_scratch(void** ptr, cudaStream_t stream);
+// The calling thread's current driver context (nullptr if none).
+cudaError_t current_context(CUcontext* ctx);
 cudaError_t read_and_clear_status(unsigned long long* out);
 
 cudaError_t launch_fwd_fp8(const Fp8FwdParams& prm, int grid, cudaStream_t stream);

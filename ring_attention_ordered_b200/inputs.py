@@ -112,6 +112,24 @@ WORKLOADS = {
 # eight ring blocks of 16K tokens.
 HEADLINE = "l128k_h32_causal"
 
+# Reduced cases for hardware-counter captures: the headline workload with a
+# quarter of its heads (K and V still 512 MiB, well past L2, so the forward
+# keeps its K/V-head-major order; about 1 GiB on the device).  Heads are
+# independent and processed one K/V head after another, so a launch's DRAM
+# traffic scales with the head count.
+PROFILE_WORKLOADS = {
+    "l128k_h8_causal": Workload(
+        "l128k_h8_causal", B=1, Hq=8, Hkv=8, L=131072, d=128, n_ring=8,
+        causal=True, seed=3),
+}
+
+
+def find_workload(name: str) -> Workload:
+    """A named workload or reduced profiling case."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    return PROFILE_WORKLOADS[name]
+
 
 def make_inputs(B: int, Hq: int, Hkv: int, L: int, d: int, seed: int,
                 k_scale: float = 1.0, sink_count: int = 0,
@@ -161,3 +179,18 @@ def sample_rows(w: Workload, n: int, seed: int | None = None):
     h = (flat // w.L) % w.Hq
     r = flat % w.L
     return np.stack([b, h, r], axis=1).astype(np.int64)
+
+
+def sample_rows_per_head(w: Workload, n: int, seed: int | None = None):
+    """``n`` distinct rows of every (b, h), each drawn uniformly without
+    replacement from one ``numpy.random.default_rng(seed)`` (default: the
+    workload's seed) taken in (b, h) order; int64 array [B * Hq * n, 3]."""
+    import numpy as np
+
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    out = []
+    for b in range(w.B):
+        for h in range(w.Hq):
+            r = rng.choice(w.L, size=min(n, w.L), replace=False)
+            out.append(np.stack([np.full_like(r, b), np.full_like(r, h), r], axis=1))
+    return np.concatenate(out).astype(np.int64)

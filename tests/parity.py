@@ -1,13 +1,26 @@
 """Comparison helpers shared by the GPU parity tests.
 
-Tolerances (fp64 oracle vs the bf16-in / fp32-accumulate / bf16-out kernel):
+Tolerances (fp64 oracle vs the bf16-in / fp32-accumulate / bf16-out kernel).
+The stated contract is max |err| <= 1e-2 and mean |err| <= 1e-3 on O and
+max |err| <= 1e-3 on LSE.
 
-* O: mean |err| <= 1e-3 over all compared elements, and per element
-  |err| <= 1e-2, widened to one bf16 ulp of the oracle value where that ulp is
-  larger (|O| >= 2): the output is stored in bf16, whose spacing there exceeds
-  1e-2, so no bf16 value can be closer than half an ulp and fp32 accumulation
-  error may round to the neighbouring value.
+* O per element: |err| <= 1e-2 wherever a bf16 value can meet it, i.e.
+  wherever half a bf16 ulp of the exact value is below 1e-2 (|O| < 4).  At
+  |O| >= 4 half an ulp is 2^-6 = 0.0156, so no stored value is within 1e-2
+  of every real number there.  The bound there is half an ulp plus O_SLACK
+  (5e-3), the kernel's own allowance before storage.  An emulation of the
+  kernel's arithmetic over all 134M output elements of the 32K GQA workload
+  gave at most 4.8e-3 before storage: fp32 accumulation, and P rounded to
+  bf16 for the P V product with O normalised by the sum of the rounded P.
+* O mean |err| <= 1e-3 over all compared elements.
 * LSE: max |err| <= 1e-3.
+
+Every comparison also records the storage floor: the error of the fp64
+oracle itself rounded to bf16 (nearest even).  It also records how many
+elements exceed 1e-2 and whether each such element lies within its floor plus
+O_SLACK.  An element over 1e-2 that does is a tolerance-spec case, not a
+kernel error.  ``parity_records()`` returns these per comparison, and the
+test session prints them as a table at the end (``conftest.py``).
 """
 
 from __future__ import annotations
@@ -18,6 +31,14 @@ import torch
 O_MAX = 1e-2
 O_MEAN = 1e-3
 LSE_MAX = 1e-3
+O_SLACK = 5e-3
+
+_RECORDS: list = []
+
+
+def parity_records() -> list:
+    """Statistics of every ``compare`` call made in this process."""
+    return list(_RECORDS)
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
@@ -27,8 +48,18 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
 
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """fp64 -> nearest bf16 value (ties to even), returned as fp64.  Scaling
+    by a power of two and rounding to an integer are exact in fp64, so this
+    is a single correct rounding (no detour through fp32)."""
+    x = np.asarray(x, dtype=np.float64)
+    u = bf16_ulp(x)
+    return np.where(x != 0, np.round(x / u) * u, 0.0)
+
+
 def o_bound(o_ref: np.ndarray) -> np.ndarray:
-    return np.maximum(O_MAX, bf16_ulp(o_ref))
+    half = 0.5 * bf16_ulp(o_ref)
+    return np.where(half < O_MAX, O_MAX, half + O_SLACK)
 
 
 def to_np(t) -> np.ndarray:
@@ -38,7 +69,7 @@ def to_np(t) -> np.ndarray:
 
 
 def compare(o_gpu, lse_gpu, o_ref, lse_ref, what: str = ""):
-    """Assert the tolerances above; return a dict of error statistics."""
+    """Assert the tolerances above; record and return error statistics."""
     og, lg = to_np(o_gpu), to_np(lse_gpu)
     o_ref = np.asarray(o_ref, dtype=np.float64)
     lse_ref = np.asarray(lse_ref, dtype=np.float64)
@@ -48,19 +79,46 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what: str = ""):
     assert np.all(np.isfinite(lg)), f"{what}: non-finite LSE"
     err = np.abs(og - o_ref)
     lerr = np.abs(lg - lse_ref)
+    floor = np.abs(round_bf16(o_ref) - o_ref)
     bound = o_bound(o_ref)
+    over = err > O_MAX
     stats = {
+        "what": what,
+        "n": int(err.size),
+        "rows": int(lerr.size),
         "o_max": float(err.max()) if err.size else 0.0,
         "o_mean": float(err.mean()) if err.size else 0.0,
-        "o_over_1e-2": int((err > O_MAX).sum()),
         "lse_max": float(lerr.max()) if lerr.size else 0.0,
-        "n": int(err.size),
+        "floor_max": float(floor.max()) if floor.size else 0.0,
+        "floor_mean": float(floor.mean()) if floor.size else 0.0,
+        "o_over_1e-2": int(over.sum()),
+        # elements over 1e-2 that lie within their storage floor + O_SLACK
+        "over_1e-2_within_floor": int((over & (err <= floor + O_SLACK)).sum()),
+        "ref_absmax": float(np.abs(o_ref).max()) if o_ref.size else 0.0,
     }
+    _RECORDS.append(stats)
     bad = err > bound
     assert not bad.any(), (
         f"{what}: {int(bad.sum())} O elements beyond bound; worst err {err[bad].max():.3e} "
         f"at ref {o_ref[bad][np.argmax(err[bad])]:.4f}; stats {stats}")
     assert stats["o_mean"] <= O_MEAN, f"{what}: mean |err| {stats['o_mean']:.3e}; {stats}"
+    assert stats["lse_max"] <= LSE_MAX, f"{what}: LSE err {stats['lse_max']:.3e}; {stats}"
+    return stats
+
+
+def compare_lse(lse_gpu, lse_ref, what: str = ""):
+    """LSE alone (a complete LSE vector against a stored oracle result):
+    max |err| <= LSE_MAX; recorded like ``compare``."""
+    lg = to_np(lse_gpu).reshape(-1)
+    lr = np.asarray(lse_ref, dtype=np.float64).reshape(-1)
+    assert lg.shape == lr.shape, (lg.shape, lr.shape)
+    assert np.all(np.isfinite(lg)), f"{what}: non-finite LSE"
+    lerr = np.abs(lg - lr)
+    stats = {"what": what, "n": 0, "rows": int(lerr.size), "o_max": None, "o_mean": None,
+             "lse_max": float(lerr.max()), "lse_mean": float(lerr.mean()),
+             "floor_max": None, "floor_mean": None, "o_over_1e-2": None,
+             "over_1e-2_within_floor": None, "ref_absmax": None}
+    _RECORDS.append(stats)
     assert stats["lse_max"] <= LSE_MAX, f"{what}: LSE err {stats['lse_max']:.3e}; {stats}"
     return stats
 

@@ -24,6 +24,7 @@ element
 
 and, for the mean over elements, the root-sum-square of the same terms
 bounds the expected error of a sum of independent zero-mean roundings.
+
 The bounds use R over every tile of the head, which is at least the R any
 kernel schedule takes, so they hold for either choice.
 """
@@ -57,7 +58,8 @@ def bounds_from_scores(s, vv, f, rel_normal: float = REL_NORMAL,
 
 
 def fp8_reference(q8, sq, k8, sk, v8, sv, causal: bool, scale: float, bhr=None,
-                  rel_normal: float = REL_NORMAL, abs_subnormal: float = ABS_SUBNORMAL):
+                  rel_normal: float = REL_NORMAL, abs_subnormal: float = ABS_SUBNORMAL,
+                  row_block: int = 256):
     """Oracle O and lse of the dequantised tensors for the rows ``bhr``
     ([n, 3] of (b, h, r); every row when None), with the per-element bounds
     ``bmax`` (worst case) and ``brms`` (root sum of squares).
@@ -86,8 +88,8 @@ def fp8_reference(q8, sq, k8, sk, v8, sv, causal: bool, scale: float, bhr=None,
         kk = k[b, :, kh, :]
         vv = v[b, :, kh, :]
         f = sv[b, kh, np.arange(L) // BLOCK] / sv[b, kh].max()
-        for s0 in range(0, len(idx), 256):
-            sel = idx[s0:s0 + 256]
+        for s0 in range(0, len(idx), row_block):
+            sel = idx[s0:s0 + row_block]
             rs = bhr[sel, 2]
             s = scale * (q[b, rs, h, :] @ kk.T)
             if causal:

@@ -193,3 +193,32 @@ def test_autograd_function_matches_oracle(ra):
     ref = oracle.attention_bwd(q, k, v, do, True, scale)
     for g_, r_, n in zip((qd.grad, kd.grad, vd.grad), ref, "qkv"):
         compare_grad(g_, r_, f"autograd d{n}")
+
+
+def test_side_stream_calls_match_the_current_stream(ra):
+    """fwd and bwd launched on a side stream, with their outputs and the
+    backward's workspace allocated by the wrapper, give bitwise the results of
+    the same calls on the current stream.  Right after the calls return, the
+    current stream allocates and fills buffers of the workspace's size: had
+    the workspace been allocated on the current stream, the caching allocator
+    could hand its block to them while the side stream's kernels still use it."""
+    from ring_attention_ordered_b200.inputs import make_grad_output, make_inputs
+    B, Hq, Hkv, L, d, n_ring = 1, 8, 2, 4096, 128, 4
+    q, k, v = (t.cuda() for t in make_inputs(B, Hq, Hkv, L, d, seed=51))
+    do = make_grad_output(B, L, Hq, d, 51).cuda()
+    out0, lse0 = ra.fwd(q, k, v, n_ring, True)
+    ref = ra.bwd(q, k, v, out0, do, lse0, n_ring, True)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    out1, lse1 = ra.fwd(q, k, v, n_ring, True, stream=side)
+    got = ra.bwd(q, k, v, out1, do, lse1, n_ring, True, stream=side)
+    ws_bytes = B * Hq * L * 4
+    junk = [torch.full((ws_bytes // 4,), float("nan"), device="cuda") for _ in range(8)]
+    side.synchronize()
+    torch.cuda.synchronize()
+    ra.check_status(side)
+    assert torch.equal(out1, out0) and torch.equal(lse1, lse0)
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    del junk

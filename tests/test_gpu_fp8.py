@@ -162,6 +162,53 @@ def test_fwd_fp8_workload_sampled_rows(ra, name, n_sample):
     assert dev.mean() < 3e-2
 
 
+def test_fwd_fp8_sink_workload_sampled_rows(ra):
+    """The 1M-token GQA workload whose first four keys carry +3 (attention
+    sinks: rows dominated by a few keys, where the E4M3 rounding of a large
+    weight matters most), 128 rows drawn per head plus sink-dominated early
+    rows and ring-block edges, against exact attention of the dequantised
+    inputs.  The oracle quantises K and V whole and Q only in the 128-row
+    tiles that hold checked rows (a tile's codes depend on that tile alone);
+    the GPU's codes of those tiles must equal the oracle's bit for bit."""
+    from oracle.fp8_fp64 import BLOCK
+    from ring_attention_ordered_b200.inputs import WORKLOADS, sample_rows_per_head, workload_inputs
+    w = WORKLOADS["l1m_gqa4_sink_causal"]
+    q, k, v = workload_inputs(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    q8, sq = ra.quantize_fp8(qd)
+    k8, sk = ra.quantize_fp8(kd)
+    v8, sv = ra.quantize_fp8(vd)
+    del qd, kd, vd
+    out, lse = ra.fwd_fp8(q8, sq, k8, sk, v8, sv, w.n_ring, w.causal, w.scale)
+    ra.check_status()
+    blk = w.L // w.n_ring
+    extra = np.array([[0, h, r] for h in (0, w.Hq - 1)
+                      for r in (0, 3, 4, 5, 17, 127, 128, 1000, blk - 1, blk, w.L - 1)])
+    bhr = np.concatenate([sample_rows_per_head(w, 128), extra]).astype(np.int64)
+    k8o, sko = quantize_blocks(k)
+    v8o, svo = quantize_blocks(v)
+    assert np.array_equal(k8.cpu().numpy(), k8o) and np.array_equal(sk.cpu().numpy(), sko)
+    assert np.array_equal(v8.cpu().numpy(), v8o) and np.array_equal(sv.cpu().numpy(), svo)
+    q8o = np.zeros(tuple(q.shape), dtype=np.uint8)
+    sqo = np.ones(tuple(sq.shape), dtype=np.float32)
+    for b, h, t in sorted({(int(b), int(h), int(r) // BLOCK) for b, h, r in bhr}):
+        c, sc = quantize_blocks(q[b:b + 1, t * BLOCK:(t + 1) * BLOCK, h:h + 1])
+        q8o[b, t * BLOCK:(t + 1) * BLOCK, h] = c[0, :, 0]
+        sqo[b, h, t] = sc[0, 0, 0]
+    for b, h, t in sorted({(int(b), int(h), int(r) // BLOCK) for b, h, r in bhr}):
+        assert np.array_equal(q8[b, t * BLOCK:(t + 1) * BLOCK, h].cpu().numpy(),
+                              q8o[b, t * BLOCK:(t + 1) * BLOCK, h])
+        assert float(sq[b, h, t]) == float(sqo[b, h, t])
+    ref = fp8_reference(q8o, sqo, k8o, sko, v8o, svo, w.causal, w.scale, bhr, row_block=32)
+    b, h, r = (torch.from_numpy(bhr[:, i]).cuda() for i in range(3))
+    stats = compare_fp8(out[b, r, h, :].float().cpu().numpy(), lse[b, h, r].cpu().numpy(), ref,
+                        w.name)
+    o_true, _ = oracle.attention_rows(q, k, v, w.causal, w.scale, bhr, row_block=16)
+    dev = np.abs(out[b, r, h, :].float().cpu().numpy() - o_true)
+    print(w.name, stats, "vs bf16-input attention: max", dev.max(), "mean", dev.mean())
+    assert dev.mean() < 3e-2
+
+
 def test_fp8_bounded_wait_reports_timeout_and_recovers(ra):
     from ring_attention_ordered_b200 import _lib
     from ring_attention_ordered_b200.inputs import make_inputs

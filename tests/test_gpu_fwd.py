@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from parity import compare, to_np
+from parity import compare, compare_lse, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -95,26 +95,66 @@ def boundary_rows(w, heads):
                     dtype=np.int64)
 
 
-@pytest.mark.parametrize("name,n_sample", [
-    ("l32k_gqa4_causal", 2048),
-    ("l128k_h32_causal", 1024),
-    ("l1m_gqa4_sink_causal", 512),
-])
-def test_workload_sampled_rows(ra, name, n_sample):
-    from ring_attention_ordered_b200.inputs import WORKLOADS, sample_rows, workload_inputs
+def _run_workload(ra, name):
+    from ring_attention_ordered_b200.inputs import WORKLOADS, workload_inputs
     w = WORKLOADS[name]
     q, k, v = workload_inputs(w)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     out, lse = ra.fwd(qd, kd, vd, w.n_ring, w.causal, w.scale)
     ra.check_status()
     del qd, kd, vd
-    bhr = np.concatenate([sample_rows(w, n_sample),
-                          boundary_rows(w, [0, w.Hq - 1])])
-    o_ref, l_ref = oracle.attention_rows(q, k, v, w.causal, w.scale, bhr)
+    return w, (q, k, v), out, lse
+
+
+def _check_rows(w, qkv, out, lse, bhr, what):
+    from oracle_pool import attention_rows_parallel
+    o_ref, l_ref = attention_rows_parallel(*qkv, w.causal, w.scale, bhr)
     b, h, r = (torch.from_numpy(bhr[:, i]).cuda() for i in range(3))
-    o_g = out[b, r, h, :]
-    l_g = lse[b, h, r]
-    compare(o_g, l_g, o_ref, l_ref, name)
+    compare(out[b, r, h, :], lse[b, h, r], o_ref, l_ref, what)
+
+
+def test_workload_l32k_gqa4_causal_all_rows(ra):
+    """Every row of every head of the GQA 32K workload (K x2: sharp peaks)."""
+    w, qkv, out, lse = _run_workload(ra, "l32k_gqa4_causal")
+    rows = np.arange(w.L, dtype=np.int64)
+    bhr = np.array([[b, h, 0] for b in range(w.B) for h in range(w.Hq)], dtype=np.int64)
+    bhr = np.repeat(bhr, w.L, axis=0)
+    bhr[:, 2] = np.tile(rows, w.B * w.Hq)
+    _check_rows(w, qkv, out, lse, bhr, f"{w.name} all {len(bhr)} rows")
+
+
+def test_workload_l128k_h32_causal_rows_and_full_lse(ra, golden_dir):
+    """The headline workload: 4096 rows drawn uniformly (every element of O
+    and the LSE), rows around every ring-block boundary of the first and last
+    head, and the complete LSE of heads 0 and 1 against the stored oracle
+    result (written by tests/golden/make_l128k_lse.py)."""
+    import hashlib
+    import json
+    import os
+    from ring_attention_ordered_b200.inputs import sample_rows
+    w, qkv, out, lse = _run_workload(ra, "l128k_h32_causal")
+    # complete LSE of heads 0 and 1
+    meta = json.load(open(os.path.join(golden_dir, "l128k_h32_causal_lse_h01.json")))
+    ref = np.load(os.path.join(golden_dir, "l128k_h32_causal_lse_h01.npy"))
+    assert hashlib.sha256(ref.tobytes()).hexdigest() == meta["array_sha256"]
+    q, k, v = qkv
+    digest = hashlib.sha256()
+    for hd in meta["heads"]:
+        for t, i in ((q, hd), (k, hd // w.group), (v, hd // w.group)):
+            digest.update(t[:, :, i].contiguous().view(torch.int16).numpy().tobytes())
+    assert digest.hexdigest() == meta["inputs_sha256"], "inputs differ from the stored ones"
+    compare_lse(lse[0, meta["heads"]], ref, f"{w.name} complete LSE of heads {meta['heads']}")
+    bhr = np.concatenate([sample_rows(w, 4096), boundary_rows(w, [0, w.Hq - 1])])
+    _check_rows(w, qkv, out, lse, bhr, f"{w.name} 4096 uniform + boundary rows")
+
+
+def test_workload_l1m_gqa4_sink_causal_rows_per_head(ra):
+    """The 1M-token sink workload: 1024 rows drawn per head (8192), plus rows
+    around every ring-block boundary of the first and last head."""
+    from ring_attention_ordered_b200.inputs import sample_rows_per_head
+    w, qkv, out, lse = _run_workload(ra, "l1m_gqa4_sink_causal")
+    bhr = np.concatenate([sample_rows_per_head(w, 1024), boundary_rows(w, [0, w.Hq - 1])])
+    _check_rows(w, qkv, out, lse, bhr, f"{w.name} 1024 rows per head + boundary rows")
 
 
 def test_special_zero_query_and_zero_scale(ra):
