@@ -24,9 +24,9 @@
 //     O_w += P_w V with P_w read from TMEM;
 //   * warps 0-3 and 4-7 each own one query tile (one TMEM lane = one row):
 //     they read S, apply the mask, keep the running max/sum in fp32, write P
-//     as bf16 back over S, rescale O in TMEM only when the running max grew by
-//     more than 2^8 (the final division cancels a stale max exactly), and run
-//     the epilogue O / l, lse = m + ln l.  The two tiles ping-pong, so one
+//     as bf16 back over S, rescale O in TMEM whenever the running max grows
+//     (so the key holding it has P = 1 exactly), and run the epilogue
+//     O / l, lse = m + ln l.  The two tiles ping-pong, so one
 //     tile's softmax runs under the other tile's MMAs (the overlap the
 //     FlashAttention article describes for FlashAttention-3);
 //   * every mbarrier wait is bounded by %globaltimer; a wait that runs out
@@ -64,7 +64,13 @@ constexpr int SOFTMAX_REGS = 224;
 constexpr int CONTROL_REGS = 56;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
-constexpr float RESCALE_LOG2 = 8.0f;
+// The reference maximum follows the row's running maximum exactly: O and l
+// are rescaled whenever a tile raises it.  The key holding the maximum then
+// has P = 2^0 = 1 exactly in bf16, so a row dominated by one key carries no
+// rounding of that key's weight into O (a lagging reference, such as one
+// moved only past 2^8, leaves P in (1, 256] there and its bf16 rounding,
+// up to 2^-9 relative, shows in O).
+constexpr float RESCALE_LOG2 = 0.0f;
 constexpr float LN2 = 0.69314718055994530942f;
 
 // Device status word: 0 = ok, otherwise (code << 32) | where.
@@ -362,23 +368,19 @@ drain:
 
 // ------------------------------------------------------------------ softmax
 // One score row (128 columns held in sr): P = 2^(s * c2 - m) written as bf16
-// pairs to TMEM columns [0, 64) at tS.  Returns the row sums of the fp32 P
-// (x, for the log-sum-exp) and of the bf16-rounded P that the P V product
-// uses (y, which normalises O, so that O is exactly the weighted mean of the
-// V rows under the rounded weights).  Arrives on p_half_bar once the first
-// 64 keys of P are stored.
+// pairs to TMEM columns [0, 64) at tS, returns the row sum of the fp32 P.
+// Arrives on p_half_bar once the first 64 keys of P are stored.
 // MASKED: columns > lim are excluded (set to zero exactly).  Issues
 // warp-collective tcgen05.st: every lane of the warp must call the same
 // instantiation at the same time.
 template <bool MASKED>
-__device__ __forceinline__ float2 exp_row_store(uint32_t (&sr)[128], float c2, float m, int lim,
-                                                uint32_t tS, uint32_t p_half_bar) {
+__device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, float m, int lim,
+                                               uint32_t tS, uint32_t p_half_bar) {
   const uint64_t c2x2 = f2_pack(c2, c2);
   const uint64_t nm2 = f2_pack(-m, -m);
-  uint64_t acc[4], accr[2];
+  uint64_t acc[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
-  accr[0] = accr[1] = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     uint32_t pk[32];
@@ -397,8 +399,6 @@ __device__ __forceinline__ float2 exp_row_store(uint32_t (&sr)[128], float c2, f
       }
       acc[j & 3] = f2_add(acc[j & 3], f2_pack(p0, p1));
       pk[j] = pack_bf16x2(p0, p1);
-      accr[j & 1] = f2_add(accr[j & 1], f2_pack(__uint_as_float(pk[j] << 16),
-                                                __uint_as_float(pk[j] & 0xffff0000u)));
     }
     tmem_st32(tS + 32 * half, pk);
     if (half == 0) {
@@ -410,10 +410,9 @@ __device__ __forceinline__ float2 exp_row_store(uint32_t (&sr)[128], float c2, f
   }
   const uint64_t s01 = f2_add(acc[0], acc[1]);
   const uint64_t s23 = f2_add(acc[2], acc[3]);
-  float a, b, ar, br;
+  float a, b;
   f2_unpack(f2_add(s01, s23), a, b);
-  f2_unpack(f2_add(accr[0], accr[1]), ar, br);
-  return make_float2(a + b, ar + br);
+  return a + b;
 }
 
 // Epilogue of a per-visit launch: this visit's normalised rows O / l (fp32)
@@ -485,9 +484,8 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
     const int qt = w ? x.qt[1] : x.qt[0];
     const int h = w ? x.h[1] : x.h[0];
     const int qrow = qt * BM + t;                  // row inside the ring block
-    // running max m (log2 units); row sums of the unrounded P (l, for the
-    // lse) and of the bf16-rounded P (lr, for O)
-    float m = -INFINITY, l = 0.f, lr = 0.f;
+    // running max m (log2 units) and row sum l of P
+    float m = -INFINITY, l = 0.f;
     KvIter it;
     it.start(p, x);
 
@@ -543,8 +541,9 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
       const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_tile = (rmax == -INFINITY) ? -INFINITY : rmax * c2;
-      // Lazy rescale: move the reference max only when the tile max exceeds
-      // it by more than 2^8 (the final O / l cancels a stale max exactly).
+      // Rescale when the tile maximum exceeds the reference (the decision is
+      // per row; the O round trip in TMEM runs for the warp when any of its
+      // rows needs it, with alpha = 1 for the others).
       const bool need = m_tile > m + RESCALE_LOG2;
       float alpha = 1.f;
       if (__any_sync(0xffffffffu, need)) {
@@ -566,10 +565,9 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
         }
         m = m_new;
       }
-      const float2 rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS, br.p_half(w))
-                                 : exp_row_store<false>(sr, c2, m, lim, tS, br.p_half(w));
-      l = l * alpha + rsum.x;
-      lr = lr * alpha + rsum.y;
+      const float rsum = masked ? exp_row_store<true>(sr, c2, m, lim, tS, br.p_half(w))
+                                : exp_row_store<false>(sr, c2, m, lim, tS, br.p_half(w));
+      l = l * alpha + rsum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(br.p_full(w));
@@ -582,11 +580,11 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
       tc_fence_after();
       const bool row_ok = qrow < p.blk_len;
       const long long pos = static_cast<long long>(x.blk) * p.blk_len + qrow;
-      const float inv_l = 1.f / lr;
+      const float inv_l = 1.f / l;
       if (p.o_acc != nullptr) {
         // a row with no allowed key (strict diagonal, row 0) is an empty
         // partial: o = 0, lse = -inf, which the fold ignores
-        visit_epilogue<D>(p, tO, row_ok, x.b, pos, h, lr > 0.f ? inv_l : 0.f, (m + log2f(l)) * LN2);
+        visit_epilogue<D>(p, tO, row_ok, x.b, pos, h, l > 0.f ? inv_l : 0.f, (m + log2f(l)) * LN2);
         tc_fence_before();
         mbar_arrive(br.o_free(w));
         ++units_w;

@@ -10,8 +10,8 @@ max |err| <= 1e-3 on LSE.
   of every real number there.  The bound there is half an ulp plus O_SLACK
   (5e-3), the kernel's own allowance before storage.  An emulation of the
   kernel's arithmetic over all 134M output elements of the 32K GQA workload
-  gave at most 4.8e-3 before storage: fp32 accumulation, and P rounded to
-  bf16 for the P V product with O normalised by the sum of the rounded P.
+  gave at most 3.0e-3 before storage: fp32 accumulation, P rounded to bf16
+  for the P V product, the reference maximum following the running maximum.
 * O mean |err| <= 1e-3 over all compared elements.
 * LSE: max |err| <= 1e-3.
 

@@ -34,6 +34,30 @@ def _bf16(shape, seed, mult=1.0):
 
 
 # ------------------------------------------------------------------ quantiser
+def _all_magnitudes_case():
+    """Tiles that hold every finite bf16 magnitude up to a chosen maximum,
+    with both signs, each tile also holding that maximum (so it sets every
+    tile's scale), for maxima at the edges of the quantiser's division: a
+    scale amax / 448 that is subnormal (IEEE division path), barely normal,
+    one and near the largest bf16."""
+    bits = np.arange(0x8000, dtype=np.uint32)
+    mags = (bits << 16).view(np.float32)
+    mags = mags[np.isfinite(mags)]
+    per_tile = 128 * 128 - 1
+    tiles = []
+    for target in (1e-37, 2.4e-35, 1.0, 3.0e38):
+        amax = np.float32(torch.tensor(target).to(torch.bfloat16).float().item())
+        m = np.sort(mags[mags <= amax])
+        vals = np.concatenate([m, -m])
+        vals = np.concatenate([vals, np.zeros(-vals.size % per_tile, dtype=np.float32)])
+        for chunk in vals.reshape(-1, per_tile):
+            tiles.append(np.concatenate([np.float32([amax]), chunk]).reshape(128, 128))
+    x = np.concatenate(tiles)[None, :, None, :]
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    assert torch.equal(xt.float(), torch.from_numpy(x))      # exact bf16 values
+    return xt
+
+
 def _quant_case(name):
     if name == "ragged_d64":
         return _bf16((1, 300, 2, 64), 1)
@@ -49,11 +73,13 @@ def _quant_case(name):
         return _bf16((1, 129, 2, 8), 4, mult=50.0)
     if name == "one_row":
         return _bf16((1, 1, 1, 16), 5)
+    if name == "all_magnitudes":
+        return _all_magnitudes_case()
     raise KeyError(name)
 
 
 @pytest.mark.parametrize("name", ["ragged_d64", "zero_and_large_tiles", "d256_two_tiles", "d8",
-                                  "one_row"])
+                                  "one_row", "all_magnitudes"])
 def test_quantize_matches_oracle_bitwise(ra, name):
     x = _quant_case(name)
     codes, scales = ra.quantize_fp8(x.cuda())
