@@ -9,9 +9,12 @@
 // remaining rows.
 //
 // One CTA per (tile, head, batch), 256 threads: a first pass of 16-byte loads
-// reduces |x| to the tile's maximum, a second pass reads the tile again (an
-// L2 hit) and writes the codes (8 bytes per store) and the scale.  The kernel
-// is bound by HBM: 2 bytes read and 1 byte written per element.
+// reduces |x| to the tile's maximum (packed bf16 maxima), a second pass
+// reads the tile again (an L2 hit) and writes the codes (8 bytes per store)
+// and the scale.  The algorithmic traffic is 2 bytes read and 1 byte written
+// per element; the instruction count per element is kept low (chunk
+// indices from compile-time shifts for d = 64, 128 and 256, packed f32x2
+// arithmetic for the quotient) so that issue does not bound the kernel.
 //
 // The quotient x / s is formed without a division per element (Markstein's
 // method for correctly rounded division): once per tile, s is scaled by a
@@ -29,6 +32,7 @@
 
 #include <cstdint>
 
+#include "ptx_sm100.cuh"
 #include "ra_internal.h"
 
 namespace ra {
@@ -44,10 +48,19 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Elementwise max of |x| over the 8 bf16 values of a chunk, on packed pairs.
+__device__ __forceinline__ __nv_bfloat162 absmax8(uint4 v, __nv_bfloat162 m) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = __hmax2(m, __habs2(h[i]));
+  return m;
+}
+
 // x / s as described in the file comment: c = 2^-e for s = 2^e (1 + f),
-// s1 = s c, r1 = 1/s1 rounded to nearest.
+// s1 = s c, r1 = 1/s1 rounded to nearest; pairs hold the same value twice.
 struct Divisor {
-  float s, c, s1, r1;
+  float s;
+  uint64_t c2, s1n2, r12;
   bool fast;
 };
 
@@ -56,31 +69,38 @@ __device__ __forceinline__ Divisor make_divisor(float s) {
   d.s = s;
   d.fast = s >= 1.17549435e-38f;   // normal float
   const uint32_t ef = (__float_as_uint(s) >> 23) & 0xffu;
-  d.c = __uint_as_float((254u - ef) << 23);
-  d.s1 = s * d.c;
-  d.r1 = __frcp_rn(d.s1);
+  const float c = __uint_as_float((254u - ef) << 23);
+  const float s1 = s * c;
+  const float r1 = __frcp_rn(s1);
+  d.c2 = f2_pack(c, c);
+  d.s1n2 = f2_pack(-s1, -s1);
+  d.r12 = f2_pack(r1, r1);
   return d;
 }
 
-__device__ __forceinline__ float quotient(float x, const Divisor& d) {
-  if (!d.fast) return __fdiv_rn(x, d.s);
-  const float x1 = x * d.c;
-  const float q0 = __fmul_rn(x1, d.r1);
-  // the sign of x: a quotient too small for E4M3 must round to the zero of
-  // x's sign, which the correction step can lose when it returns zero
-  return copysignf(fmaf(fmaf(-q0, d.s1, x1), d.r1, q0), x);
-}
-
-__device__ __forceinline__ float absmax8(uint4 v, float m) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+// E4M3 codes of two bf16 values (a bf16x2 word) divided by the scale.
+__device__ __forceinline__ uint32_t quantize_pair(uint32_t xb, const Divisor& d) {
+  const float x0 = __uint_as_float(xb << 16);
+  const float x1 = __uint_as_float(xb & 0xffff0000u);
+  float q0, q1;
+  if (d.fast) {
+    const uint64_t xs = f2_mul(f2_pack(x0, x1), d.c2);        // exact: power-of-two scaling
+    const uint64_t p = f2_mul(xs, d.r12);
+    const uint64_t q = f2_fma(f2_fma(p, d.s1n2, xs), d.r12, p);
+    f2_unpack(q, q0, q1);
+    // the sign of x: a quotient too small for E4M3 must round to the zero
+    // of x's sign, which the correction step can lose when it returns zero
+    q0 = copysignf(q0, x0);
+    q1 = copysignf(q1, x1);
+  } else {
+    q0 = __fdiv_rn(x0, d.s);
+    q1 = __fdiv_rn(x1, d.s);
   }
-  return m;
+  return e4m3x2(q0, q1);
 }
 
+// CPR: 16-byte chunks per row (d / 8) when known at compile time, else 0.
+template <int CPR>
 __global__ void __launch_bounds__(QT) ra_quant_fp8_kernel(const __nv_bfloat16* __restrict__ x,
                                                           uint8_t* __restrict__ codes,
                                                           float* __restrict__ scales, long long L,
@@ -89,21 +109,23 @@ __global__ void __launch_bounds__(QT) ra_quant_fp8_kernel(const __nv_bfloat16* _
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long r0 = static_cast<long long>(t) * ROWS;
   const int rows = static_cast<int>(min(static_cast<long long>(ROWS), L - r0));
-  const int cpr = d / 8;                         // 16-byte chunks per row
+  const int cpr = CPR ? CPR : d / 8;             // 16-byte chunks per row
   const int n = rows * cpr;
   const long long row_stride = static_cast<long long>(H) * d;
   const long long base = (static_cast<long long>(b) * L + r0) * row_stride + static_cast<long long>(h) * d;
+  constexpr int NCH = CPR ? (ROWS * CPR + QT - 1) / QT : MAX_CHUNKS;
 
   // pass 1: the tile's maximum magnitude (loads only, all in flight at once)
-  float m = 0.f;
+  __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
 #pragma unroll
-  for (int i = 0; i < MAX_CHUNKS; ++i) {
+  for (int i = 0; i < NCH; ++i) {
     const int c = threadIdx.x + i * QT;
     if (c < n) {
       const int r = c / cpr, cc = c % cpr;
-      m = absmax8(__ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc), m);
+      m2 = absmax8(__ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc), m2);
     }
   }
+  float m = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -116,24 +138,16 @@ __global__ void __launch_bounds__(QT) ra_quant_fp8_kernel(const __nv_bfloat16* _
   if (threadIdx.x == 0) scales[(static_cast<long long>(b) * H + h) * T + t] = s;
 
   // pass 2: read the tile again (from L2: it was read a moment ago) and
-  // write the codes.  Holding the tile in registers between the passes
-  // instead would cut the resident CTAs per SM from 8 to 3.
+  // write the codes.
 #pragma unroll 4
-  for (int i = 0; i < MAX_CHUNKS; ++i) {
+  for (int i = 0; i < NCH; ++i) {
     const int c = threadIdx.x + i * QT;
     if (c < n) {
       const int r = c / cpr, cc = c % cpr;
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + base + r * row_stride) + cc);
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
-      uint32_t w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(hv[j]);
-        w[j] = e4m3x2(quotient(f.x, dv), quotient(f.y, dv));
-      }
       uint2 out;
-      out.x = w[0] | (w[1] << 16);
-      out.y = w[2] | (w[3] << 16);
+      out.x = quantize_pair(v.x, dv) | (quantize_pair(v.y, dv) << 16);
+      out.y = quantize_pair(v.z, dv) | (quantize_pair(v.w, dv) << 16);
       *(reinterpret_cast<uint2*>(codes + base + r * row_stride) + cc) = out;
     }
   }
@@ -147,7 +161,15 @@ cudaError_t launch_quantize_fp8(const __nv_bfloat16* x, uint8_t* codes, float* s
   if (T > 0x7fffffffll || H > 65535 || B > 65535) return cudaErrorInvalidValue;
   if (d % 8 != 0 || d < 8 || d > 256) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>(H), static_cast<unsigned>(B));
-  ra_quant_fp8_kernel<<<grid, QT, 0, stream>>>(x, codes, scales, L, H, d, static_cast<int>(T));
+  const int Ti = static_cast<int>(T);
+  if (d == 128)
+    ra_quant_fp8_kernel<16><<<grid, QT, 0, stream>>>(x, codes, scales, L, H, d, Ti);
+  else if (d == 64)
+    ra_quant_fp8_kernel<8><<<grid, QT, 0, stream>>>(x, codes, scales, L, H, d, Ti);
+  else if (d == 256)
+    ra_quant_fp8_kernel<32><<<grid, QT, 0, stream>>>(x, codes, scales, L, H, d, Ti);
+  else
+    ra_quant_fp8_kernel<0><<<grid, QT, 0, stream>>>(x, codes, scales, L, H, d, Ti);
   return cudaGetLastError();
 }
 
