@@ -107,6 +107,7 @@ class ClockSampler:
 
 
 KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd.cu",
+                  "ring_attention_ordered_b200/csrc/ra_fwd_roles.cuh",
                   "ring_attention_ordered_b200/csrc/ptx_sm100.cuh",
                   "ring_attention_ordered_b200/csrc/ra_api.cu",
                   "ring_attention_ordered_b200/csrc/ra_internal.h",
@@ -114,6 +115,7 @@ KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd.cu",
                   "ring_attention_ordered_b200/csrc/ra_sync.cuh",
                   "ring_attention_ordered_b200/csrc/ra_schedule.cuh"]
 FP8_KERNEL_SOURCES = ["ring_attention_ordered_b200/csrc/ra_fwd_fp8.cu",
+                      "ring_attention_ordered_b200/csrc/ra_fwd_roles.cuh",
                       "ring_attention_ordered_b200/csrc/ptx_sm100.cuh",
                       "ring_attention_ordered_b200/csrc/ra_api.cu",
                       "ring_attention_ordered_b200/csrc/ra_internal.h",

@@ -72,6 +72,40 @@ cudaError_t current_context(CUcontext* ctx) {
   return fn(ctx) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
 }
 
+cudaError_t symbol_address(const void* symbol, void** ptr, cudaStream_t stream) {
+  struct Entry {
+    CUcontext ctx;
+    const void* symbol;
+    void* addr;
+  };
+  static std::mutex mu;
+  static Entry cache[64] = {};
+  static int n_cached = 0;
+  CUcontext ctx = nullptr;
+  cudaError_t e = current_context(&ctx);
+  if (e != cudaSuccess) return e;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  int slot = -1;
+  for (int i = 0; i < n_cached; ++i)
+    if (cache[i].ctx == ctx && cache[i].symbol == symbol) slot = i;
+  if (cs == cudaStreamCaptureStatusNone || slot < 0 || ctx == nullptr) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, symbol);
+    if (e != cudaSuccess) return e;
+    // the lookup made a context current if there was none
+    if (ctx == nullptr && (e = current_context(&ctx)) != cudaSuccess) return e;
+    for (int i = 0; i < n_cached; ++i)
+      if (cache[i].ctx == ctx && cache[i].symbol == symbol) slot = i;
+    if (slot < 0) slot = (n_cached < 64) ? n_cached++ : 0;
+    cache[slot] = Entry{ctx, symbol, addr};
+  }
+  *ptr = cache[slot].addr;
+  return cudaSuccess;
+}
+
 }  // namespace ra
 
 namespace {
@@ -210,7 +244,9 @@ ra_status launch_forward(const void* q, const void* k, const void* v, void* out,
   const int cap = g_max_ctas.load();
   if (cap > 0 && cap < grid) grid = cap;
   if (grid > prm.total_units) grid = prm.total_units;
-  cudaError_t e = ra::launch_fwd(prm, d, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = ra::next_ticket_counter(reinterpret_cast<cudaStream_t>(stream), &prm.tickets);
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "work queue reset: %s", cudaGetErrorString(e));
+  e = ra::launch_fwd(prm, d, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "forward launch: %s", cudaGetErrorString(e));
   return ok();
 }
@@ -617,7 +653,9 @@ ra_status ring_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, cons
   const int cap = g_max_ctas.load();
   if (cap > 0 && cap < grid) grid = cap;
   if (grid > prm.total_units) grid = prm.total_units;
-  cudaError_t e = ra::launch_fwd_fp8(prm, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = ra::next_ticket_counter(reinterpret_cast<cudaStream_t>(stream), &prm.tickets);
+  if (e != cudaSuccess) return fail(RA_ERR_CUDA, "work queue reset: %s", cudaGetErrorString(e));
+  e = ra::launch_fwd_fp8(prm, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(RA_ERR_CUDA, "FP8 forward launch: %s", cudaGetErrorString(e));
   return ok();
 }

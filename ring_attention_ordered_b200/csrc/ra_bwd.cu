@@ -1128,36 +1128,7 @@ cudaError_t launch_bwd(const BwdParams& prm, int d, int num_sms, int max_ctas,
 __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchRows];
 
 cudaError_t noalloc_scratch(void** ptr, cudaStream_t stream) {
-  struct Entry {
-    CUcontext ctx;
-    void* addr;
-  };
-  static std::mutex mu;
-  static Entry cache[64] = {};
-  static int n_cached = 0;
-  CUcontext ctx = nullptr;
-  cudaError_t e = current_context(&ctx);
-  if (e != cudaSuccess) return e;
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  e = cudaStreamIsCapturing(stream, &cs);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lk(mu);
-  int slot = -1;
-  for (int i = 0; i < n_cached; ++i)
-    if (cache[i].ctx == ctx) slot = i;
-  if (cs == cudaStreamCaptureStatusNone || slot < 0 || ctx == nullptr) {
-    void* addr = nullptr;
-    e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    // the lookup made a context current if there was none
-    if (ctx == nullptr && (e = current_context(&ctx)) != cudaSuccess) return e;
-    for (int i = 0; i < n_cached; ++i)
-      if (cache[i].ctx == ctx) slot = i;
-    if (slot < 0) slot = (n_cached < 64) ? n_cached++ : 0;
-    cache[slot] = Entry{ctx, addr};
-  }
-  *ptr = cache[slot].addr;
-  return cudaSuccess;
+  return symbol_address(reinterpret_cast<const void*>(&g_noalloc_scratch), ptr, stream);
 }
 
 cudaError_t read_and_clear_bwd_status(unsigned long long* out) {

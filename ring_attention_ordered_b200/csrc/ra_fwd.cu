@@ -13,11 +13,13 @@
 //   * grouped-query heads share K/V tiles (lnwmold page §2.2).
 //
 // How (B200 design):
-//   * persistent CTAs, one per SM, each owning a static, snake-ordered share
-//     of work units sorted longest-first (the causal load balance of L4 §4.5,
-//     limitation 3); a unit is two 128-row query tiles that see the same K/V
-//     stream -- two heads of one GQA group at the same rows, or two adjacent
-//     tiles of one head inside one ring block;
+//   * persistent CTAs, one per SM, taking work units from a queue shared by
+//     the launch (an atomic counter over units sorted longest first, the
+//     causal load balance of L4 §4.5, limitation 3), so that all CTAs stay
+//     within about one unit of each other and the K/V heads they read stay
+//     few; a unit is two 128-row query tiles that see the same K/V stream --
+//     two heads of one GQA group at the same rows, or two adjacent tiles of
+//     one head inside one ring block;
 //   * warp 8 loads Q/K/V tiles with TMA (128-byte swizzle) into a K/V ring of
 //     shared-memory stages;
 //   * warp 9 (one thread) issues tcgen05.mma: S_w = Q_w K^T into TMEM, then
@@ -36,10 +38,12 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 
 #include "ptx_sm100.cuh"
+#include "ra_fwd_roles.cuh"
 #include "ra_internal.h"
 #include "ra_merge_math.cuh"
 #include "ra_schedule.cuh"
@@ -48,8 +52,8 @@
 
 namespace ra {
 
-constexpr int BM = 128;             // query rows per tile
-constexpr int BN = 128;             // keys per K/V tile
+constexpr int BM = FWD_BM;          // query rows per tile
+constexpr int BN = FWD_BN;          // keys per K/V tile
 constexpr int BOX_COLS = 64;        // TMA box width (64 bf16 = one 128-byte swizzle row)
 constexpr int BOX_BYTES = 128 * 128;
 constexpr int NUM_THREADS = 384;   // three warpgroups
@@ -76,11 +80,11 @@ constexpr float LN2 = 0.69314718055994530942f;
 // Device status word: 0 = ok, otherwise (code << 32) | where.
 __device__ unsigned long long g_ra_status = 0ull;
 
-enum WaitSite : uint32_t {
-  SITE_Q_FULL = 1, SITE_Q_EMPTY, SITE_KV_FULL, SITE_KV_EMPTY, SITE_S_FULL,
-  SITE_P_FULL, SITE_O_DONE, SITE_O_FREE, SITE_P_HALF
-};
+// Work-queue counters of the forward launches (see next_ticket_counter).
+__device__ unsigned int g_ra_tickets[kTicketSlots];
 
+// Shared-memory layout (D = head dim): Q0, Q1, NS K/V stages, barriers, the
+// TMEM holder and abort flag, the unit queue.
 template <int D>
 struct Cfg {
   static constexpr int Q_BYTES = BM * D * 2;
@@ -89,99 +93,11 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  // barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2],
-  // p_full[2], o_done[2], o_free[2], p_half[2], drain; then tmem holder +
-  // abort flag
-  static constexpr int NUM_BARS = 2 + 2 * NS + 10 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int OFF_MISC = OFF_BAR + fwd_num_bars(NS) * 8;
+  static constexpr int OFF_UNITS = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_UNITS + UQ * 4 + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
-
-struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, o_done0, o_free0, p_half0, drain;
-  __device__ __forceinline__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
-  __device__ __forceinline__ uint32_t kv_empty(int s) const { return kv_empty0 + 8u * s; }
-  __device__ __forceinline__ uint32_t s_full(int w) const { return s_full0 + 8u * w; }
-  __device__ __forceinline__ uint32_t p_full(int w) const { return p_full0 + 8u * w; }
-  __device__ __forceinline__ uint32_t o_done(int w) const { return o_done0 + 8u * w; }
-  __device__ __forceinline__ uint32_t o_free(int w) const { return o_free0 + 8u * w; }
-  __device__ __forceinline__ uint32_t p_half(int w) const { return p_half0 + 8u * w; }
-};
-
-// ------------------------------------------------------------------ loader
-// The whole warp runs the control flow, so every address and coordinate is
-// warp-uniform (uniform registers); lane 0 alone issues the copies.
-template <int D>
-__device__ void loader_role(const FwdParams& p, const Bars& br, uint32_t smem_base, const Ctl& cx) {
-  using C = Cfg<D>;
-  constexpr int NBOX = D / BOX_COLS;
-  const bool leader = (threadIdx.x & 31) == 0;
-  const int G = gridDim.x, c = blockIdx.x;
-  uint32_t kv_it = 0, q_uses = 0;
-  bool q_pending = false;
-  for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.total_units) break;
-    const Unit x = decode_unit(p, u);
-    if (q_uses > 0 && !wait_warp(br.q_empty, (q_uses - 1) & 1u, cx, SITE_Q_EMPTY)) goto drain;
-    if ((p.debug_flags & 1u) && q_uses == 0) {
-      // fault injection: the first query tiles are never requested
-    } else {
-      const int nq = x.valid1 ? 2 : 1;
-      const int row0 = x.b * p.L + x.blk * p.blk_len;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(br.q_full, nq * C::Q_BYTES);
-#pragma unroll
-        for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d(smem_base + C::OFF_Q + bx * BOX_BYTES, &p.tm_q, br.q_full, bx * BOX_COLS,
-                      x.h[0], row0 + x.qt[0] * BM);
-        if (x.valid1) {
-#pragma unroll
-          for (int bx = 0; bx < NBOX; ++bx)
-            tma_load_3d(smem_base + C::OFF_Q + C::Q_BYTES + bx * BOX_BYTES, &p.tm_q, br.q_full,
-                        bx * BOX_COLS, x.h[1], row0 + x.qt[1] * BM);
-        }
-      }
-      __syncwarp();
-      q_pending = true;
-    }
-    ++q_uses;
-    KvIter it;
-    it.start(p, x);
-    for (int idx = 0; idx < x.n_kv; ++idx, it.next(p)) {
-      const int row = x.b * p.L + it.jb * p.blk_len + it.kl * BN;
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        const int s = kv_it % C::NS;
-        const uint32_t ph = (kv_it / C::NS) & 1u;
-        if (!wait_warp(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
-        const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(br.kv_full(s), C::KV_BYTES);
-#pragma unroll
-          for (int bx = 0; bx < NBOX; ++bx)
-            tma_load_3d(smem_base + C::OFF_KV + s * C::KV_BYTES + bx * BOX_BYTES, map,
-                        br.kv_full(s), bx * BOX_COLS, x.kvh, row);
-        }
-        __syncwarp();
-        ++kv_it;
-      }
-    }
-  }
-  return;
-drain:
-  // Let the copies already issued land before the CTA's shared memory goes.
-  if (leader) {
-    const uint32_t n = kv_it < static_cast<uint32_t>(C::NS) ? kv_it : C::NS;
-    for (uint32_t i = 0; i < n; ++i) {
-      const uint32_t it = kv_it - 1 - i;
-      drain_wait(br.kv_full(it % C::NS), (it / C::NS) & 1u, 200000000ull);
-    }
-    if (q_pending) drain_wait(br.q_full, (q_uses - 1) & 1u, 200000000ull);
-  }
-  __syncwarp();
-}
 
 // ------------------------------------------------------------------ MMA
 template <int KK>
@@ -220,151 +136,63 @@ __device__ __forceinline__ void mma_pv_half(uint32_t d, uint32_t p_tmem, uint32_
   if (elect_one()) mma_ts<C0 + 24, B0 + 384>(d, p_tmem, b, hi, idesc, 1u);
 }
 
+// Geometry of the bf16 kernel for the shared loader and MMA roles: a tile
+// row of D bf16 values is D / 64 TMA boxes of 64 columns (one 128-byte
+// swizzle row each), BOX_BYTES apart; tcgen05.mma kind::f16 with K = 16.
 template <int D>
-__device__ void mma_role(const FwdParams& p, const Bars& br, uint32_t smem_base, uint32_t tmem,
-                         const Ctl& cx) {
+struct Bf16Geom {
   using C = Cfg<D>;
-  constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false);
-  constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
-  const bool leader = (threadIdx.x & 31) == 0;
-  const int G = gridDim.x, c = blockIdx.x;
-  uint32_t kv_it = 0, q_uses = 0;
-  uint32_t pf_phase0 = 0u, pf_phase1 = 0u;
-  uint32_t units0 = 0u, units1 = 0u;
+  static constexpr int Q_BYTES = C::Q_BYTES;
+  static constexpr int KV_BYTES = C::KV_BYTES;
+  static constexpr int NS = C::NS;
+  static constexpr int OFF_Q = C::OFF_Q;
+  static constexpr int OFF_KV = C::OFF_KV;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
+
+  static __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map,
+                                                   uint32_t bar, int h, int row) {
+#pragma unroll
+    for (int bx = 0; bx < D / BOX_COLS; ++bx)
+      tma_load_3d(dst + bx * BOX_BYTES, map, bar, bx * BOX_COLS, h, row);
+  }
+  static __device__ __forceinline__ void load_q(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                int h, int row) {
+    load_tile(dst, map, bar, h, row);
+  }
+  static __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int h, int row) {
+    load_tile(dst, map, bar, h, row);
+  }
 
   // Shared-memory descriptors as (low, high) words.  The start address sits
   // in the low 14 bits in 16-byte units; every offset used here keeps the
   // address below 2^18 bytes, so adding (offset >> 4) to the low word never
   // carries out of that field.  The high words are fixed by the layout.
-  const uint64_t dq0 = smem_desc_sw128(smem_base + C::OFF_Q, 16, 1024);
-  const uint64_t dkv0 = smem_desc_sw128(smem_base + C::OFF_KV, 16, 1024);
-  const uint64_t dv0 = smem_desc_sw128(smem_base + C::OFF_KV, BOX_BYTES, 1024);
-  const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dkv0);
-  const uint32_t v_lo = static_cast<uint32_t>(dv0);
-  const uint32_t k_hi = static_cast<uint32_t>(dkv0 >> 32), v_hi = static_cast<uint32_t>(dv0 >> 32);
-  auto issue_qk = [&](int w, int stage) {
-    const uint32_t a = q_lo + ((w * C::Q_BYTES) >> 4);
-    const uint32_t b = k_lo + ((stage * C::KV_BYTES) >> 4);
-    const uint32_t d = tmem + w * 128;
-    // k-steps of 16 elements: 32 bytes apart inside a 64-column swizzle
-    // box, the next box BOX_BYTES further on
-    mma_qk_steps<D>(d, a, b, k_hi, IDESC_QK);
-  };
-  auto issue_pv_half = [&](int w, int stage, int half, bool acc) {
-    const uint32_t b = v_lo + ((stage * C::KV_BYTES) >> 4);
-    if (half == 0)
-      mma_pv_half<0>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u);
-    else
-      mma_pv_half<1>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, 1u);
-  };
-  auto commit = [&](uint32_t bar) {
-    if (elect_one()) tc_commit(bar);
-  };
-
-  for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.total_units) break;
-    const Unit x = decode_unit(p, u);
-    const int n = x.n_kv;
-    if (!wait_warp(br.q_full, q_uses & 1u, cx, SITE_Q_FULL)) goto drain;
-    tc_fence_after();
-    ++q_uses;
-    {
-      const int ks = kv_it % C::NS;
-      if (!wait_warp(br.kv_full(ks), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
-      tc_fence_after();
-      issue_qk(0, ks);
-      commit(br.s_full(0));
-      if (x.valid1) {
-        issue_qk(1, ks);
-        commit(br.s_full(1));
-      }
-      commit(br.kv_empty(ks));
-      ++kv_it;
-      if (n == 1) commit(br.q_empty);
-    }
-    // Barrier states probed ahead of time: a probe issued before a batch of
-    // MMAs overlaps its latency with their issue, and a barrier found
-    // complete is not waited on again.
-    bool rdy_v = false, rdy_k = false, rdy_p0 = false;
-    for (int idx = 0; idx < n; ++idx) {
-      const bool more = idx + 1 < n;
-      const int vs = kv_it % C::NS;
-      const int ks = (kv_it + 1) % C::NS;
-      if (!rdy_v && !wait_warp(br.kv_full(vs), (kv_it / C::NS) & 1u, cx, SITE_KV_FULL)) goto drain;
-      // the next K tile is needed right after P0 V: wait for it now, off the
-      // softmax -> MMA -> softmax chain
-      if (more && !rdy_k &&
-          !wait_warp(br.kv_full(ks), ((kv_it + 1) / C::NS) & 1u, cx, SITE_KV_FULL))
-        goto drain;
-      tc_fence_after();
-      // query tile 0: P0 V in two halves as P0 arrives, then S0 for the next
-      // K/V tile
-      if (idx == 0 && units0 > 0) {
-        if (!wait_warp(br.o_free(0), (units0 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
-      }
-      if (!rdy_p0 && !wait_warp(br.p_half(0), pf_phase0, cx, SITE_P_HALF)) goto drain;
-      tc_fence_after();
-      issue_pv_half(0, vs, 0, idx > 0);
-      if (!wait_warp(br.p_full(0), pf_phase0, cx, SITE_P_FULL)) goto drain;
-      pf_phase0 ^= 1u;
-      tc_fence_after();
-      issue_pv_half(0, vs, 1, true);
-      if (!more) commit(br.o_done(0));
-      // probe P1's first half now; the vote on the result comes after the
-      // S0 MMAs, so the probe's latency overlaps their issue
-      const bool raw_p1 = x.valid1 ? mbar_test_wait(br.p_half(1), pf_phase1) : true;
-      if (more) {
-        issue_qk(0, ks);
-        commit(br.s_full(0));
-      }
-      const bool rdy_p1 = __all_sync(0xffffffffu, raw_p1);
-      // query tile 1
-      if (x.valid1) {
-        if (idx == 0 && units1 > 0) {
-          if (!wait_warp(br.o_free(1), (units1 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
-        }
-        if (!rdy_p1 && !wait_warp(br.p_half(1), pf_phase1, cx, SITE_P_HALF)) goto drain;
-        tc_fence_after();
-        issue_pv_half(1, vs, 0, idx > 0);
-        if (!wait_warp(br.p_full(1), pf_phase1, cx, SITE_P_FULL)) goto drain;
-        pf_phase1 ^= 1u;
-        tc_fence_after();
-        issue_pv_half(1, vs, 1, true);
-        if (!more) commit(br.o_done(1));
-      }
-      // V of this step has been read by every P V issued so far
-      commit(br.kv_empty(vs));
-      if (more) {
-        // probe what the next step needs, then issue S1 for it
-        const bool raw_v =
-            mbar_test_wait(br.kv_full((kv_it + 2) % C::NS), ((kv_it + 2) / C::NS) & 1u);
-        const bool raw_k =
-            idx + 2 < n
-                ? mbar_test_wait(br.kv_full((kv_it + 3) % C::NS), ((kv_it + 3) / C::NS) & 1u)
-                : true;
-        const bool raw_p0 = mbar_test_wait(br.p_half(0), pf_phase0);
-        if (x.valid1) {
-          issue_qk(1, ks);
-          commit(br.s_full(1));
-        }
-        rdy_v = __all_sync(0xffffffffu, raw_v);
-        rdy_k = __all_sync(0xffffffffu, raw_k);
-        rdy_p0 = __all_sync(0xffffffffu, raw_p0);
-        commit(br.kv_empty(ks));
-        if (idx + 1 == n - 1) commit(br.q_empty);
-      }
-      kv_it += more ? 2u : 1u;
-    }
-    ++units0;
-    if (x.valid1) ++units1;
+  uint32_t q_lo, k_lo, v_lo, k_hi, v_hi;
+  __device__ explicit Bf16Geom(uint32_t smem_base) {
+    const uint64_t dq0 = smem_desc_sw128(smem_base + OFF_Q, 16, 1024);
+    const uint64_t dkv0 = smem_desc_sw128(smem_base + OFF_KV, 16, 1024);
+    const uint64_t dv0 = smem_desc_sw128(smem_base + OFF_KV, BOX_BYTES, 1024);
+    q_lo = static_cast<uint32_t>(dq0);
+    k_lo = static_cast<uint32_t>(dkv0);
+    v_lo = static_cast<uint32_t>(dv0);
+    k_hi = static_cast<uint32_t>(dkv0 >> 32);
+    v_hi = static_cast<uint32_t>(dv0 >> 32);
   }
-  return;
-drain:
-  commit(br.drain);
-  if (leader) drain_wait(br.drain, 0u, 200000000ull);
-  __syncwarp();
-}
+  // S_w = Q_w K^T into TMEM at d: k-steps of 16 elements, 32 bytes apart
+  // inside a 64-column swizzle box, the next box BOX_BYTES further on.
+  __device__ __forceinline__ void issue_qk(uint32_t d, int w, int stage) const {
+    mma_qk_steps<D>(d, q_lo + ((w * Q_BYTES) >> 4), k_lo + ((stage * KV_BYTES) >> 4), k_hi,
+                    IDESC_QK);
+  }
+  // O_w (+)= P_w V over keys 64 HALF .. 64 HALF + 63.
+  template <int HALF>
+  __device__ __forceinline__ void issue_pv_half(uint32_t d, uint32_t p_tmem, int stage,
+                                                uint32_t acc) const {
+    mma_pv_half<HALF>(d, p_tmem, v_lo + ((stage * KV_BYTES) >> 4), v_hi, IDESC_PV, acc);
+  }
+};
 
 // ------------------------------------------------------------------ softmax
 // One score row (128 columns held in sr): P = 2^(s * c2 - m) written as bf16
@@ -465,7 +293,7 @@ __device__ __forceinline__ void visit_epilogue(const FwdParams& p, uint32_t tO, 
 }
 
 template <int D>
-__device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, int w,
+__device__ void softmax_role(const FwdParams& p, const FwdBars& br, uint32_t tmem, int w,
                              const Ctl& cx) {
   const int t = threadIdx.x - w * 128;            // row inside the query tile
   const int quarter = (threadIdx.x >> 5) & 3;     // TMEM lane quarter of this warp
@@ -473,12 +301,14 @@ __device__ void softmax_role(const FwdParams& p, const Bars& br, uint32_t tmem, 
   const uint32_t tS = tmem + lane_off + w * 128;  // S (fp32) and P (bf16 pairs, first 64 cols)
   const uint32_t tO = tmem + lane_off + 256 + w * 128;
   const float c2 = p.scale_log2;
-  const int G = gridDim.x, cta = blockIdx.x;
   uint32_t s_phase = 0u, units_w = 0u;
 
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, cta);
-    if (u >= p.total_units) break;
+    int u;
+    const bool got = next_unit(br, k, cx, u);
+    if (!__all_sync(0xffffffffu, got)) return;
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u < 0) break;
     const Unit x = decode_unit(p, u);
     if (w == 1 && !x.valid1) continue;
     const int qt = w ? x.qt[1] : x.qt[0];
@@ -625,37 +455,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_fwd_kernel(const __grid_con
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
 
-  Bars br;
-  br.q_full = base + C::OFF_BAR;
-  br.q_empty = br.q_full + 8;
-  br.kv_full0 = br.q_empty + 8;
-  br.kv_empty0 = br.kv_full0 + 8 * C::NS;
-  br.s_full0 = br.kv_empty0 + 8 * C::NS;
-  br.p_full0 = br.s_full0 + 16;
-  br.o_done0 = br.p_full0 + 16;
-  br.o_free0 = br.o_done0 + 16;
-  br.p_half0 = br.o_free0 + 16;
-  br.drain = br.p_half0 + 16;
+  FwdBars br;
+  br.layout(base + C::OFF_BAR, C::NS, base + C::OFF_UNITS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(br.q_full, 1);
-    mbar_init(br.q_empty, 1);
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(br.kv_full(s), 1);
-      mbar_init(br.kv_empty(s), 1);
-    }
-    for (int w = 0; w < 2; ++w) {
-      mbar_init(br.s_full(w), 1);
-      mbar_init(br.p_full(w), 128);
-      mbar_init(br.o_done(w), 1);
-      mbar_init(br.o_free(w), 128);
-      mbar_init(br.p_half(w), 128);
-    }
-    mbar_init(br.drain, 1);
+    br.init(C::NS);
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
@@ -680,9 +488,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_fwd_kernel(const __grid_con
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(CONTROL_REGS));
     if (warp == WARP_LOAD) {
-      loader_role<D>(p, br, base, cx);
+      fwd_loader_role<Bf16Geom<D>>(p, br, base, cx);
     } else if (warp == WARP_MMA) {
-      mma_role<D>(p, br, base, tmem, cx);
+      fwd_mma_role<Bf16Geom<D>>(p, br, base, tmem, cx);
     }
   }
 
@@ -723,6 +531,18 @@ static cudaError_t launch_fwd_d(const FwdParams& prm, int grid, cudaStream_t str
 cudaError_t launch_fwd(const FwdParams& prm, int d, int grid, cudaStream_t stream) {
   if (d == 128) return launch_fwd_d<128>(prm, grid, stream);
   return launch_fwd_d<64>(prm, grid, stream);
+}
+
+cudaError_t next_ticket_counter(cudaStream_t stream, unsigned int** counter) {
+  static std::atomic<unsigned> next{0u};
+  void* base = nullptr;
+  cudaError_t e = symbol_address(reinterpret_cast<const void*>(&g_ra_tickets), &base, stream);
+  if (e != cudaSuccess) return e;
+  unsigned int* slot = static_cast<unsigned int*>(base) + (next.fetch_add(1u) % kTicketSlots);
+  e = cudaMemsetAsync(slot, 0, sizeof(unsigned int), stream);
+  if (e != cudaSuccess) return e;
+  *counter = slot;
+  return cudaSuccess;
 }
 
 cudaError_t read_and_clear_status(unsigned long long* out) {

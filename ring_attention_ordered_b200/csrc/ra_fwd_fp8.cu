@@ -22,8 +22,10 @@
 //     the epilogue multiplies O by R / l;
 //   * tiles are 16 KB: one TMA box (128 rows x 128 bytes, 128-byte swizzle)
 //     per tile and 8 K/V stages; V is read as an MN-major B operand.
-//   Roles, barriers, lazy rescale (threshold 2^8, so P' <= 256 stays below
-//   E4M3's 448) and bounded waits are those of the bf16 kernel.
+//   The loader and MMA roles, the work queue and the barriers are the bf16
+//   kernel's (ra_fwd_roles.cuh, with this kernel's tile geometry); the
+//   softmax keeps a lazy rescale (threshold 2^8, so P' <= 256 stays below
+//   E4M3's 448).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,6 +33,7 @@
 #include <cstdint>
 
 #include "ptx_sm100.cuh"
+#include "ra_fwd_roles.cuh"
 #include "ra_internal.h"
 #include "ra_schedule.cuh"
 #include "ra_sync.cuh"
@@ -39,8 +42,8 @@
 namespace ra {
 namespace fp8 {
 
-constexpr int BM = 128;
-constexpr int BN = 128;
+constexpr int BM = FWD_BM;
+constexpr int BN = FWD_BN;
 constexpr int D = 128;
 constexpr int TILE_BYTES = 128 * 128;   // 128 rows x 128 E4M3 values
 constexpr int NUM_THREADS = 384;
@@ -58,90 +61,14 @@ constexpr int NS = 8;                         // K/V stages
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
-// barriers: q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], p_full[2],
-// o_done[2], o_free[2], p_half[2], drain; then tmem holder + abort flag
-constexpr int NUM_BARS = 2 + 2 * NS + 10 + 1;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;   // + alignment slack
+// barriers (ra_fwd_roles.cuh), then tmem holder + abort flag, then the unit
+// queue
+constexpr int OFF_MISC = OFF_BAR + fwd_num_bars(NS) * 8;
+constexpr int OFF_UNITS = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_UNITS + UQ * 4 + 1024;   // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 __device__ unsigned long long g_status = 0ull;
-
-enum WaitSite : uint32_t {
-  SITE_Q_FULL = 1, SITE_Q_EMPTY, SITE_KV_FULL, SITE_KV_EMPTY, SITE_S_FULL,
-  SITE_P_FULL, SITE_O_DONE, SITE_O_FREE, SITE_P_HALF
-};
-
-struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, o_done0, o_free0, p_half0, drain;
-  __device__ __forceinline__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
-  __device__ __forceinline__ uint32_t kv_empty(int s) const { return kv_empty0 + 8u * s; }
-  __device__ __forceinline__ uint32_t s_full(int w) const { return s_full0 + 8u * w; }
-  __device__ __forceinline__ uint32_t p_full(int w) const { return p_full0 + 8u * w; }
-  __device__ __forceinline__ uint32_t o_done(int w) const { return o_done0 + 8u * w; }
-  __device__ __forceinline__ uint32_t o_free(int w) const { return o_free0 + 8u * w; }
-  __device__ __forceinline__ uint32_t p_half(int w) const { return p_half0 + 8u * w; }
-};
-
-// ------------------------------------------------------------------ loader
-__device__ void loader_role(const Fp8FwdParams& p, const Bars& br, uint32_t smem_base,
-                            const Ctl& cx) {
-  const bool leader = (threadIdx.x & 31) == 0;
-  const int G = gridDim.x, c = blockIdx.x;
-  uint32_t kv_it = 0, q_uses = 0;
-  bool q_pending = false;
-  for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.total_units) break;
-    const Unit x = decode_unit(p, u);
-    if (q_uses > 0 && !wait_warp(br.q_empty, (q_uses - 1) & 1u, cx, SITE_Q_EMPTY)) goto drain;
-    if ((p.debug_flags & 1u) && q_uses == 0) {
-      // fault injection: the first query tiles are never requested
-    } else {
-      const int nq = x.valid1 ? 2 : 1;
-      const int row0 = x.b * p.L + x.blk * p.blk_len;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(br.q_full, nq * TILE_BYTES);
-        tma_load_3d(smem_base + OFF_Q, &p.tm_q, br.q_full, 0, x.h[0], row0 + x.qt[0] * BM);
-        if (x.valid1)
-          tma_load_3d(smem_base + OFF_Q + TILE_BYTES, &p.tm_q, br.q_full, 0, x.h[1],
-                      row0 + x.qt[1] * BM);
-      }
-      __syncwarp();
-      q_pending = true;
-    }
-    ++q_uses;
-    KvIter it;
-    it.start(p, x);
-    for (int idx = 0; idx < x.n_kv; ++idx, it.next(p)) {
-      const int row = x.b * p.L + it.jb * p.blk_len + it.kl * BN;
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        const int s = kv_it % NS;
-        const uint32_t ph = (kv_it / NS) & 1u;
-        if (!wait_warp(br.kv_empty(s), ph ^ 1u, cx, SITE_KV_EMPTY)) goto drain;
-        const CUtensorMap* map = kv ? &p.tm_v : &p.tm_k;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(br.kv_full(s), TILE_BYTES);
-          tma_load_3d(smem_base + OFF_KV + s * TILE_BYTES, map, br.kv_full(s), 0, x.kvh, row);
-        }
-        __syncwarp();
-        ++kv_it;
-      }
-    }
-  }
-  return;
-drain:
-  if (leader) {
-    const uint32_t n = kv_it < static_cast<uint32_t>(NS) ? kv_it : NS;
-    for (uint32_t i = 0; i < n; ++i) {
-      const uint32_t it = kv_it - 1 - i;
-      drain_wait(br.kv_full(it % NS), (it / NS) & 1u, 200000000ull);
-    }
-    if (q_pending) drain_wait(br.q_full, (q_uses - 1) & 1u, 200000000ull);
-  }
-  __syncwarp();
-}
 
 // ------------------------------------------------------------------ MMA
 // S = Q8 K8^T: 4 MMAs of K = 32 (32 bytes apart inside the 128-byte swizzle
@@ -165,132 +92,51 @@ __device__ __forceinline__ void mma_pv_half(uint32_t d, uint32_t p_tmem, uint32_
   if (elect_one()) mma_ts_f8<C0 + 8, B0 + 256>(d, p_tmem, b, hi, idesc, 1u);
 }
 
-__device__ void mma_role(const Fp8FwdParams& p, const Bars& br, uint32_t smem_base, uint32_t tmem,
-                         const Ctl& cx) {
-  constexpr uint32_t IDESC_QK = idesc_e4m3_f32(BM, BN, false);
-  constexpr uint32_t IDESC_PV = idesc_e4m3_f32(BM, D, true);
-  const bool leader = (threadIdx.x & 31) == 0;
-  const int G = gridDim.x, c = blockIdx.x;
-  uint32_t kv_it = 0, q_uses = 0;
-  uint32_t pf_phase0 = 0u, pf_phase1 = 0u;
-  uint32_t units0 = 0u, units1 = 0u;
+// Geometry of the FP8 kernel for the shared loader and MMA roles: a tile is
+// one TMA box of 128 rows x 128 bytes (one 128-byte swizzle row per row);
+// tcgen05.mma kind::f8f6f4 with K = 32.
+struct Fp8Geom {
+  static constexpr int Q_BYTES = TILE_BYTES;
+  static constexpr int KV_BYTES = TILE_BYTES;
+  static constexpr int NS = fp8::NS;
+  static constexpr int OFF_Q = fp8::OFF_Q;
+  static constexpr int OFF_KV = fp8::OFF_KV;
+  static constexpr uint32_t IDESC_QK = idesc_e4m3_f32(BM, BN, false);
+  static constexpr uint32_t IDESC_PV = idesc_e4m3_f32(BM, D, true);
+
+  static __device__ __forceinline__ void load_q(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                int h, int row) {
+    tma_load_3d(dst, map, bar, 0, h, row);
+  }
+  static __device__ __forceinline__ void load_kv(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int h, int row) {
+    tma_load_3d(dst, map, bar, 0, h, row);
+  }
 
   // Descriptor low words (start address in 16-byte units below 2^18 bytes,
   // so added offsets never carry out of the field) and the shared high word.
   // V is MN-major: its 128 E4M3 values per key span exactly one 128-byte
   // swizzle atom along N, so the atom stride (leading byte offset) is never
   // used; it is set to 16 bytes, which keeps even a misread inside the tile.
-  const uint64_t dq0 = smem_desc_sw128(smem_base + OFF_Q, 16, 1024);
-  const uint64_t dkv0 = smem_desc_sw128(smem_base + OFF_KV, 16, 1024);
-  const uint64_t dv0 = smem_desc_sw128(smem_base + OFF_KV, 16, 1024);
-  const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dkv0);
-  const uint32_t v_lo = static_cast<uint32_t>(dv0);
-  const uint32_t k_hi = static_cast<uint32_t>(dkv0 >> 32), v_hi = static_cast<uint32_t>(dv0 >> 32);
-  auto issue_qk = [&](int w, int stage) {
-    mma_qk(tmem + w * 128, q_lo + ((w * TILE_BYTES) >> 4), k_lo + ((stage * TILE_BYTES) >> 4),
-           k_hi, IDESC_QK);
-  };
-  auto issue_pv_half = [&](int w, int stage, int half, bool acc) {
-    const uint32_t b = v_lo + ((stage * TILE_BYTES) >> 4);
-    if (half == 0)
-      mma_pv_half<0>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, acc ? 1u : 0u);
-    else
-      mma_pv_half<1>(tmem + 256 + w * 128, tmem + w * 128, b, v_hi, IDESC_PV, 1u);
-  };
-  auto commit = [&](uint32_t bar) {
-    if (elect_one()) tc_commit(bar);
-  };
-
-  for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.total_units) break;
-    const Unit x = decode_unit(p, u);
-    const int n = x.n_kv;
-    if (!wait_warp(br.q_full, q_uses & 1u, cx, SITE_Q_FULL)) goto drain;
-    tc_fence_after();
-    ++q_uses;
-    {
-      const int ks = kv_it % NS;
-      if (!wait_warp(br.kv_full(ks), (kv_it / NS) & 1u, cx, SITE_KV_FULL)) goto drain;
-      tc_fence_after();
-      issue_qk(0, ks);
-      commit(br.s_full(0));
-      if (x.valid1) {
-        issue_qk(1, ks);
-        commit(br.s_full(1));
-      }
-      commit(br.kv_empty(ks));
-      ++kv_it;
-      if (n == 1) commit(br.q_empty);
-    }
-    bool rdy_v = false, rdy_k = false, rdy_p0 = false;
-    for (int idx = 0; idx < n; ++idx) {
-      const bool more = idx + 1 < n;
-      const int vs = kv_it % NS;
-      const int ks = (kv_it + 1) % NS;
-      if (!rdy_v && !wait_warp(br.kv_full(vs), (kv_it / NS) & 1u, cx, SITE_KV_FULL)) goto drain;
-      if (more && !rdy_k &&
-          !wait_warp(br.kv_full(ks), ((kv_it + 1) / NS) & 1u, cx, SITE_KV_FULL))
-        goto drain;
-      tc_fence_after();
-      if (idx == 0 && units0 > 0) {
-        if (!wait_warp(br.o_free(0), (units0 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
-      }
-      if (!rdy_p0 && !wait_warp(br.p_half(0), pf_phase0, cx, SITE_P_HALF)) goto drain;
-      tc_fence_after();
-      issue_pv_half(0, vs, 0, idx > 0);
-      if (!wait_warp(br.p_full(0), pf_phase0, cx, SITE_P_FULL)) goto drain;
-      pf_phase0 ^= 1u;
-      tc_fence_after();
-      issue_pv_half(0, vs, 1, true);
-      if (!more) commit(br.o_done(0));
-      const bool raw_p1 = x.valid1 ? mbar_test_wait(br.p_half(1), pf_phase1) : true;
-      if (more) {
-        issue_qk(0, ks);
-        commit(br.s_full(0));
-      }
-      const bool rdy_p1 = __all_sync(0xffffffffu, raw_p1);
-      if (x.valid1) {
-        if (idx == 0 && units1 > 0) {
-          if (!wait_warp(br.o_free(1), (units1 - 1) & 1u, cx, SITE_O_FREE)) goto drain;
-        }
-        if (!rdy_p1 && !wait_warp(br.p_half(1), pf_phase1, cx, SITE_P_HALF)) goto drain;
-        tc_fence_after();
-        issue_pv_half(1, vs, 0, idx > 0);
-        if (!wait_warp(br.p_full(1), pf_phase1, cx, SITE_P_FULL)) goto drain;
-        pf_phase1 ^= 1u;
-        tc_fence_after();
-        issue_pv_half(1, vs, 1, true);
-        if (!more) commit(br.o_done(1));
-      }
-      commit(br.kv_empty(vs));
-      if (more) {
-        const bool raw_v = mbar_test_wait(br.kv_full((kv_it + 2) % NS), ((kv_it + 2) / NS) & 1u);
-        const bool raw_k =
-            idx + 2 < n ? mbar_test_wait(br.kv_full((kv_it + 3) % NS), ((kv_it + 3) / NS) & 1u)
-                        : true;
-        const bool raw_p0 = mbar_test_wait(br.p_half(0), pf_phase0);
-        if (x.valid1) {
-          issue_qk(1, ks);
-          commit(br.s_full(1));
-        }
-        rdy_v = __all_sync(0xffffffffu, raw_v);
-        rdy_k = __all_sync(0xffffffffu, raw_k);
-        rdy_p0 = __all_sync(0xffffffffu, raw_p0);
-        commit(br.kv_empty(ks));
-        if (idx + 1 == n - 1) commit(br.q_empty);
-      }
-      kv_it += more ? 2u : 1u;
-    }
-    ++units0;
-    if (x.valid1) ++units1;
+  uint32_t q_lo, k_lo, v_lo, k_hi, v_hi;
+  __device__ explicit Fp8Geom(uint32_t smem_base) {
+    const uint64_t dq0 = smem_desc_sw128(smem_base + OFF_Q, 16, 1024);
+    const uint64_t dkv0 = smem_desc_sw128(smem_base + OFF_KV, 16, 1024);
+    q_lo = static_cast<uint32_t>(dq0);
+    k_lo = static_cast<uint32_t>(dkv0);
+    v_lo = static_cast<uint32_t>(dkv0);
+    k_hi = static_cast<uint32_t>(dkv0 >> 32);
+    v_hi = static_cast<uint32_t>(dkv0 >> 32);
   }
-  return;
-drain:
-  commit(br.drain);
-  if (leader) drain_wait(br.drain, 0u, 200000000ull);
-  __syncwarp();
-}
+  __device__ __forceinline__ void issue_qk(uint32_t d, int w, int stage) const {
+    mma_qk(d, q_lo + ((w * TILE_BYTES) >> 4), k_lo + ((stage * TILE_BYTES) >> 4), k_hi, IDESC_QK);
+  }
+  template <int HALF>
+  __device__ __forceinline__ void issue_pv_half(uint32_t d, uint32_t p_tmem, int stage,
+                                                uint32_t acc) const {
+    mma_pv_half<HALF>(d, p_tmem, v_lo + ((stage * TILE_BYTES) >> 4), v_hi, IDESC_PV, acc);
+  }
+};
 
 // ------------------------------------------------------------------ softmax
 // One score row (128 columns in sr): P' = 2^(s * c2 + bias) rounded to E4M3
@@ -344,7 +190,7 @@ __device__ __forceinline__ float exp_row_store(uint32_t (&sr)[128], float c2, fl
   return a + b;
 }
 
-__device__ void softmax_role(const Fp8FwdParams& p, const Bars& br, uint32_t tmem, int w,
+__device__ void softmax_role(const Fp8FwdParams& p, const FwdBars& br, uint32_t tmem, int w,
                              const Ctl& cx) {
   const int t = threadIdx.x - w * 128;
   const int lane = threadIdx.x & 31;
@@ -352,14 +198,16 @@ __device__ void softmax_role(const Fp8FwdParams& p, const Bars& br, uint32_t tme
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tS = tmem + lane_off + w * 128;  // S (fp32), then P' (E4M3, first 32 columns)
   const uint32_t tO = tmem + lane_off + 256 + w * 128;
-  const int G = gridDim.x, cta = blockIdx.x;
   uint32_t s_phase = 0u, units_w = 0u;
   int r_head = -1;          // (batch, K/V head) whose R is cached
   float R = 1.f, log2R = 0.f;
 
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, cta);
-    if (u >= p.total_units) break;
+    int u;
+    const bool got = next_unit(br, k, cx, u);
+    if (!__all_sync(0xffffffffu, got)) return;
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u < 0) break;
     const Unit x = decode_unit(p, u);
     if (w == 1 && !x.valid1) continue;
     const int qt = w ? x.qt[1] : x.qt[0];
@@ -497,37 +345,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
 
-  Bars br;
-  br.q_full = base + OFF_BAR;
-  br.q_empty = br.q_full + 8;
-  br.kv_full0 = br.q_empty + 8;
-  br.kv_empty0 = br.kv_full0 + 8 * NS;
-  br.s_full0 = br.kv_empty0 + 8 * NS;
-  br.p_full0 = br.s_full0 + 16;
-  br.o_done0 = br.p_full0 + 16;
-  br.o_free0 = br.o_done0 + 16;
-  br.p_half0 = br.o_free0 + 16;
-  br.drain = br.p_half0 + 16;
+  FwdBars br;
+  br.layout(base + OFF_BAR, NS, base + OFF_UNITS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base_ptr + OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(br.q_full, 1);
-    mbar_init(br.q_empty, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(br.kv_full(s), 1);
-      mbar_init(br.kv_empty(s), 1);
-    }
-    for (int w = 0; w < 2; ++w) {
-      mbar_init(br.s_full(w), 1);
-      mbar_init(br.p_full(w), 128);
-      mbar_init(br.o_done(w), 1);
-      mbar_init(br.o_free(w), 128);
-      mbar_init(br.p_half(w), 128);
-    }
-    mbar_init(br.drain, 1);
+    br.init(NS);
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
@@ -552,9 +378,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(CONTROL_REGS));
     if (warp == WARP_LOAD) {
-      loader_role(p, br, base, cx);
+      fwd_loader_role<Fp8Geom>(p, br, base, cx);
     } else if (warp == WARP_MMA) {
-      mma_role(p, br, base, tmem, cx);
+      fwd_mma_role<Fp8Geom>(p, br, base, tmem, cx);
     }
   }
 

@@ -38,6 +38,9 @@ struct FwdParams {
   float scale_log2;    // scale * log2(e)
   unsigned long long wait_limit_ns;
   unsigned debug_flags;
+  // Work queue of this launch: a counter (zero at launch) from which each
+  // CTA's loader takes the next unit, in the unit order above.
+  unsigned int* tickets;
 };
 
 // Parameters of one FP8 forward launch (d = 128).  The tensor maps describe
@@ -67,6 +70,7 @@ struct Fp8FwdParams {
   float scale_log2;    // scale * log2(e), before the per-tile scales
   unsigned long long wait_limit_ns;
   unsigned debug_flags;
+  unsigned int* tickets;   // the launch's work queue (see FwdParams)
 };
 
 // Parameters of the two backward launches (dQ kernel, then dK/dV kernel).
@@ -123,7 +127,19 @@ constexpr long long kNoAllocScratchRows = 1ll << 20;
 cudaError_t noalloc_scratch(void** ptr, cudaStream_t stream);
 // The calling thread's current driver context (nullptr if none).
 cudaError_t current_context(CUcontext* ctx);
+// Device address of a static __device__ variable of this library in the
+// current context.  Looked up on every call made while `stream` is not
+// capturing (the module, and so the address, belongs to a context, which
+// cudaDeviceReset or a caller's own context can change); during a capture
+// the address last found for the current context is used.
+cudaError_t symbol_address(const void* symbol, void** ptr, cudaStream_t stream);
 cudaError_t read_and_clear_status(unsigned long long* out);
+// A zeroed work-queue counter for the next forward launch on `stream`: one of
+// kTicketSlots static device counters, taken in rotation and reset by a
+// memset ordered on the stream (so launches on different streams use
+// different counters, up to kTicketSlots at a time).
+constexpr int kTicketSlots = 64;
+cudaError_t next_ticket_counter(cudaStream_t stream, unsigned int** counter);
 
 cudaError_t launch_fwd_fp8(const Fp8FwdParams& prm, int grid, cudaStream_t stream);
 cudaError_t read_and_clear_fp8_status(unsigned long long* out);
