@@ -354,11 +354,11 @@ ra_status ring_attn_set_wait_limit_ns(uint64_t ns);
 ra_status ring_attn_set_max_ctas(int n);
 
 /* Order in which the forward kernels' persistent CTAs (bf16 and FP8) take
- * work units (a unit = two 128-row query tiles sharing one K/V stream;
- * causal units differ in length).  Results do not depend on it.
- * Process-wide.
+ * work units from the launch's queue (a unit = two 128-row query tiles
+ * sharing one K/V stream; causal units differ in length).  Results do not
+ * depend on it.  Process-wide.
  *   RA_SCHEDULE_AUTO (default): HEAD_MAJOR when the K/V tensors exceed
- *     256 MiB, else LONGEST_FIRST.
+ *     96 MiB, else LONGEST_FIRST.
  *   RA_SCHEDULE_LONGEST_FIRST: every unit sorted by length, longest first
  *     (causal load balance, "Ring Attention 环注意力" L4 §4.5 limitation 3).
  *   RA_SCHEDULE_HEAD_MAJOR: longest first within each (batch, K/V head), heads

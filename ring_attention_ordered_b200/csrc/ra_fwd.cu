@@ -27,8 +27,8 @@
 //   * warps 0-3 and 4-7 each own one query tile (one TMEM lane = one row):
 //     they read S, apply the mask, keep the running max/sum in fp32, write P
 //     as bf16 back over S, rescale O in TMEM whenever the running max grows
-//     (so the key holding it has P = 1 exactly), and run the epilogue
-//     O / l, lse = m + ln l.  The two tiles ping-pong, so one
+//     by more than a factor 2 (so a dominant key has P = 1 exactly), and run
+//     the epilogue O / l, lse = m + ln l.  The two tiles ping-pong, so one
 //     tile's softmax runs under the other tile's MMAs (the overlap the
 //     FlashAttention article describes for FlashAttention-3);
 //   * every mbarrier wait is bounded by %globaltimer; a wait that runs out
@@ -68,13 +68,15 @@ constexpr int SOFTMAX_REGS = 224;
 constexpr int CONTROL_REGS = 56;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
-// The reference maximum follows the row's running maximum exactly: O and l
-// are rescaled whenever a tile raises it.  The key holding the maximum then
-// has P = 2^0 = 1 exactly in bf16, so a row dominated by one key carries no
-// rounding of that key's weight into O (a lagging reference, such as one
-// moved only past 2^8, leaves P in (1, 256] there and its bf16 rounding,
-// up to 2^-9 relative, shows in O).
-constexpr float RESCALE_LOG2 = 0.0f;
+// The reference maximum follows the row's running maximum closely: O and l
+// are rescaled whenever a tile raises it by more than a factor 2 (1 in log2
+// units).  A key that dominates its row stands that far above the earlier
+// maximum, so it sets the reference and gets P = 2^0 = 1, exact in bf16: its
+// weight carries no bf16 rounding into O.  (A reference moved only past 2^8
+// leaves such a key's P in (1, 256], and that P's bf16 rounding, up to 2^-9
+// relative, shows in O; following every rise of the maximum costs O
+// rescales in many more steps for the same accuracy.)
+constexpr float RESCALE_LOG2 = 1.0f;
 constexpr float LN2 = 0.69314718055994530942f;
 
 // Device status word: 0 = ok, otherwise (code << 32) | where.
@@ -371,9 +373,10 @@ __device__ void softmax_role(const FwdParams& p, const FwdBars& br, uint32_t tme
       const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_tile = (rmax == -INFINITY) ? -INFINITY : rmax * c2;
-      // Rescale when the tile maximum exceeds the reference (the decision is
-      // per row; the O round trip in TMEM runs for the warp when any of its
-      // rows needs it, with alpha = 1 for the others).
+      // Rescale when the tile maximum exceeds the reference by more than
+      // RESCALE_LOG2 (the decision is per row; the O round trip in TMEM runs
+      // for the warp when any of its rows needs it, with alpha = 1 for the
+      // others; the final O / l cancels the reference exactly).
       const bool need = m_tile > m + RESCALE_LOG2;
       float alpha = 1.f;
       if (__any_sync(0xffffffffu, need)) {

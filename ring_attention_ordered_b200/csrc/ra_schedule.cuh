@@ -1,5 +1,6 @@
-// Work units of the forward kernels and their persistent schedule, shared
-// by the bf16 and FP8 forward kernels.  The parameter structs of both carry
+// Work units of the forward kernels and their order, shared by the bf16 and
+// FP8 forward kernels (which take them from a launch-wide queue in this
+// order, ra_fwd_roles.cuh).  The parameter structs of both carry
 // the same scheduling fields (B, Hq, Hkv, group, n_ring, blk_len, causal,
 // tiles_per_blk, pair_heads, head_slots, pairs_per_blk, head_major,
 // total_units), so these helpers are templates over the struct.
@@ -103,12 +104,5 @@ struct KvIter {
     }
   }
 };
-
-// Static persistent schedule: in round k, CTA c takes unit k*G + c (k even)
-// or k*G + G-1-c (k odd).  Units are sorted longest first, so the snake keeps
-// the per-CTA totals within about one unit of each other.
-__device__ __forceinline__ int unit_for_round(int k, int G, int c) {
-  return k * G + ((k & 1) ? (G - 1 - c) : c);
-}
 
 }  // namespace ra

@@ -114,11 +114,11 @@ HEADLINE = "l128k_h32_causal"
 
 # Reduced cases for hardware-counter captures: the headline workload with a
 # quarter or half of its heads.  Heads are independent and the forward runs
-# them one K/V head after another once K and V exceed 256 MiB, so a launch's
+# them one K/V head after another once K and V exceed 96 MiB, so a launch's
 # DRAM traffic scales with the head count (the two sizes check that).  With 8
-# heads the bf16 K and V are 512 MiB (about 1 GiB on the device); the FP8
-# codes of K and V reach 512 MiB only with 16 heads (about 3 GiB on the
-# device with the bf16 inputs).
+# heads the bf16 K and V are 512 MiB (about 1 GiB on the device); with 16
+# heads the FP8 codes of K and V are 512 MiB too (about 3 GiB on the device
+# with the bf16 inputs).
 PROFILE_WORKLOADS = {
     "l128k_h8_causal": Workload(
         "l128k_h8_causal", B=1, Hq=8, Hkv=8, L=131072, d=128, n_ring=8,
