@@ -45,6 +45,7 @@
 #include "ptx_sm100.cuh"
 #include "ra_internal.h"
 #include "ra_sync.cuh"
+#include "ra_unit_queue.cuh"
 #include "ring_attn.h"
 
 namespace ra {
@@ -69,12 +70,8 @@ __device__ unsigned long long g_status = 0ull;
 
 enum Site : uint32_t {
   SITE_KV_FULL = 17, SITE_KV_EMPTY, SITE_QD_FULL, SITE_QD_EMPTY, SITE_S_FULL, SITE_S_FREE,
-  SITE_DP_FULL, SITE_P_FULL, SITE_DS_FULL, SITE_ACC_DONE, SITE_ACC_FREE
+  SITE_DP_FULL, SITE_P_FULL, SITE_DS_FULL, SITE_ACC_DONE, SITE_ACC_FREE, SITE_UNIT
 };
-
-__device__ __forceinline__ int unit_for_round(int k, int G, int c) {
-  return k * G + ((k & 1) ? (G - 1 - c) : c);
-}
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
@@ -223,10 +220,12 @@ struct QCfg {
   static constexpr int OFF_V = OFF_K + NK * TILE;
   static constexpr int OFF_BAR = OFF_V + NV * TILE;
   // qo_full, qo_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
-  // s_full, s_free, dp_full, ds_full, acc_done, acc_free, drain
-  static constexpr int NUM_BARS = 2 + 2 * NK + 2 * NV + 7;
+  // s_full, s_free, dp_full, ds_full, acc_done, acc_free, drain, then the
+  // unit queue's barriers
+  static constexpr int NUM_BARS = 2 + 2 * NK + 2 * NV + 7 + UNIT_QUEUE_DEPTH;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int OFF_UNITS = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_UNITS + 4 * UNIT_QUEUE_DEPTH + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -248,6 +247,7 @@ struct QBars {
   __device__ __forceinline__ uint32_t acc_done() const { return s_full() + 32; }
   __device__ __forceinline__ uint32_t acc_free() const { return s_full() + 40; }
   __device__ __forceinline__ uint32_t drain() const { return s_full() + 48; }
+  __device__ __forceinline__ uint32_t units0() const { return s_full() + 56; }
 };
 
 struct QUnit {
@@ -288,15 +288,15 @@ struct KvWalk {
 };
 
 template <int D>
-__device__ void dq_loader(const BwdParams& p, const QBars& br, uint32_t base, const Ctl& cx) {
+__device__ void dq_loader(const BwdParams& p, const QBars& br, const UnitQueue& uq, uint32_t base,
+                          const Ctl& cx) {
   using C = QCfg<D>;
   constexpr int NBOX = D / BOX_COLS;
-  const int G = gridDim.x, c = blockIdx.x;
   uint32_t kv_it = 0, units = 0;
   bool qo_pending = false;
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.units_dq) break;
+    const int u = uq.take(p.tickets_dq, p.units_dq, k);
+    if (u < 0) break;
     const QUnit x = q_unit(p, u);
     if (units > 0 && !wait_warp(br.qo_empty(), (units - 1) & 1u, cx, SITE_QD_EMPTY)) goto drain;
     if ((p.debug_flags & 1u) && units == 0) {
@@ -363,12 +363,11 @@ drain:
 }
 
 template <int D>
-__device__ void dq_mma(const BwdParams& p, const QBars& br, uint32_t base, uint32_t tmem,
-                       const Ctl& cx) {
+__device__ void dq_mma(const BwdParams& p, const QBars& br, const UnitQueue& uq, uint32_t base,
+                       uint32_t tmem, const Ctl& cx) {
   using C = QCfg<D>;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(TM, TM, false);
   constexpr uint32_t IDESC_DQ = idesc_bf16_f32(TM, D, true);
-  const int G = gridDim.x, c = blockIdx.x;
   const uint64_t dq0 = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
   const uint64_t ddo0 = smem_desc_sw128(base + C::OFF_DO, 16, 1024);
   const uint64_t dk0 = smem_desc_sw128(base + C::OFF_K, 16, 1024);
@@ -386,8 +385,9 @@ __device__ void dq_mma(const BwdParams& p, const QBars& br, uint32_t base, uint3
     mma_kmajor<D>(t_dp, do_lo, v_lo + ((sv * C::TILE) >> 4), hi, IDESC_S);
   };
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.units_dq) break;
+    int u;
+    if (!uq.read(k, cx, SITE_UNIT, u)) goto drain;
+    if (u < 0) break;
     const QUnit x = q_unit(p, u);
     const int n = x.n;
     if (!wait_warp(br.qo_full(), units & 1u, cx, SITE_QD_FULL)) goto drain;
@@ -445,8 +445,8 @@ drain:
 }
 
 template <int D>
-__device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, int wg,
-                           const Ctl& cx) {
+__device__ void dq_softmax(const BwdParams& p, const QBars& br, const UnitQueue& uq, uint32_t tmem,
+                           int wg, const Ctl& cx) {
   constexpr int D2 = D / 2;                        // dQ columns of this warpgroup
   const int t = threadIdx.x & 127;                 // row inside the query tile
   const int quarter = (threadIdx.x >> 5) & 3;
@@ -456,11 +456,11 @@ __device__ void dq_softmax(const BwdParams& p, const QBars& br, uint32_t tmem, i
   const uint32_t t_dq = tmem + lane_off + 256 + D2 * wg;
   const int col0 = HALF * wg;
   const float c2 = p.scale_log2;
-  const int G = gridDim.x, c = blockIdx.x;
   uint32_t units = 0, step = 0;
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.units_dq) break;
+    int u;
+    if (!uq.read(k, cx, SITE_UNIT, u)) return;
+    if (u < 0) break;
     const QUnit x = q_unit(p, u);
     const int qrow = x.qt * TM + t;
     const bool valid = qrow < p.blk_len;
@@ -573,6 +573,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gen + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gen + C::OFF_MISC + 4);
   const QBars br{base + C::OFF_BAR, C::NK, C::NV};
+  // the loader runs at most two units ahead of the softmax warpgroups (it
+  // takes unit k + 2 only after the MMA warp has finished unit k's products,
+  // which needed all of unit k's dS), so the queue's four slots never overrun
+  const UnitQueue uq{br.units0(), base + C::OFF_UNITS};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     mbar_init(br.qo_full(), 1);
@@ -592,6 +596,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_
     mbar_init(br.acc_done(), 1);
     mbar_init(br.acc_free(), SOFTMAX_THREADS);
     mbar_init(br.drain(), 1);
+    uq.init();
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
@@ -611,11 +616,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dq_kernel(const __grid_
   const uint32_t tmem = *tmem_holder;
   const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
   if (warp < 8) {
-    dq_softmax<D>(p, br, tmem, warp >> 2, cx);
+    dq_softmax<D>(p, br, uq, tmem, warp >> 2, cx);
   } else if (warp == WARP_LOAD) {
-    dq_loader<D>(p, br, base, cx);
+    dq_loader<D>(p, br, uq, base, cx);
   } else {
-    dq_mma<D>(p, br, base, tmem, cx);
+    dq_mma<D>(p, br, uq, base, tmem, cx);
   }
   tc_fence_before();
   __syncthreads();
@@ -645,13 +650,15 @@ struct KCfg {
   static constexpr int OFF_DV = OFF_LSE + NQ * TM * 4;  // per dO stage: D [128]
   static constexpr int OFF_BAR = OFF_DV + NO * TM * 4;
   // kv_full, kv_empty, q_full[NQ], q_empty[NQ], do_full[NO], do_empty[NO],
-  // s_full, dp_full, s_free, pd_full, acc_done, acc_free, drain
-  static constexpr int NUM_BARS = 2 + 2 * NQ + 2 * NO + 7;
+  // s_full, dp_full, s_free, pd_full, acc_done, acc_free, drain, then the
+  // unit queue's barriers
+  static constexpr int NUM_BARS = 2 + 2 * NQ + 2 * NO + 7 + UNIT_QUEUE_DEPTH;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_UNITS = OFF_MISC + 16;
   // no alignment slack: the kernel checks that the dynamic shared memory
   // starts on a 1024-byte boundary (the 128-byte swizzle needs it) and
   // reports RA_ERR_UNSUPPORTED otherwise
-  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_UNITS + 4 * UNIT_QUEUE_DEPTH;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -673,6 +680,7 @@ struct KBars {
   __device__ __forceinline__ uint32_t acc_done() const { return s_full() + 32; }
   __device__ __forceinline__ uint32_t acc_free() const { return s_full() + 40; }
   __device__ __forceinline__ uint32_t drain() const { return s_full() + 48; }
+  __device__ __forceinline__ uint32_t units0() const { return s_full() + 56; }
 };
 
 struct KUnit {
@@ -723,17 +731,16 @@ struct QWalk {
 };
 
 template <int D>
-__device__ void kv_loader(const BwdParams& p, const KBars& br, uint32_t base, float* lse_smem,
-                          float* dv_smem, const Ctl& cx) {
+__device__ void kv_loader(const BwdParams& p, const KBars& br, const UnitQueue& uq, uint32_t base,
+                          float* lse_smem, float* dv_smem, const Ctl& cx) {
   using C = KCfg<D>;
   constexpr int NBOX = D / BOX_COLS;
   const int lane = threadIdx.x & 31;
-  const int G = gridDim.x, c = blockIdx.x;
   uint32_t q_it = 0, units = 0;
   bool kv_pending = false;
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.units_kv) break;
+    const int u = uq.take(p.tickets_kv, p.units_kv, k);
+    if (u < 0) break;
     const KUnit x = kv_unit(p, u);
     if (units > 0 && !wait_warp(br.kv_empty(), (units - 1) & 1u, cx, SITE_KV_EMPTY)) goto drain;
     {
@@ -817,12 +824,11 @@ drain:
 }
 
 template <int D>
-__device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint32_t tmem,
-                       const Ctl& cx) {
+__device__ void kv_mma(const BwdParams& p, const KBars& br, const UnitQueue& uq, uint32_t base,
+                       uint32_t tmem, const Ctl& cx) {
   using C = KCfg<D>;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(TM, TM, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16_f32(TM, D, true);
-  const int G = gridDim.x, c = blockIdx.x;
   const uint64_t dk0 = smem_desc_sw128(base + C::OFF_K, 16, 1024);
   const uint64_t dv0 = smem_desc_sw128(base + C::OFF_V, 16, 1024);
   const uint64_t dq0 = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
@@ -841,8 +847,9 @@ __device__ void kv_mma(const BwdParams& p, const KBars& br, uint32_t base, uint3
     mma_kmajor<D>(t_dp, v_lo, do_lo + ((so * C::TILE) >> 4), hi, IDESC_S);
   };
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.units_kv) break;
+    int u;
+    if (!uq.read(k, cx, SITE_UNIT, u)) goto drain;
+    if (u < 0) break;
     const KUnit x = kv_unit(p, u);
     const int n = x.n;
     if (!wait_warp(br.kv_full(), units & 1u, cx, SITE_KV_FULL)) goto drain;
@@ -907,8 +914,8 @@ drain:
 }
 
 template <int D>
-__device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, const float* lse_smem,
-                           const float* dv_smem, int wg, const Ctl& cx) {
+__device__ void kv_softmax(const BwdParams& p, const KBars& br, const UnitQueue& uq, uint32_t tmem,
+                           const float* lse_smem, const float* dv_smem, int wg, const Ctl& cx) {
   using C = KCfg<D>;
   constexpr int D2 = D / 2;                        // dK, dV columns of this warpgroup
   const int t = threadIdx.x & 127;                 // key row inside the tile
@@ -919,11 +926,11 @@ __device__ void kv_softmax(const BwdParams& p, const KBars& br, uint32_t tmem, c
   const uint32_t t_dv = tmem + lane_off + 256 + D2 * wg, t_dk = tmem + lane_off + 256 + D + D2 * wg;
   const int col0 = HALF * wg;
   const uint64_t c2x2 = f2_pack(p.scale_log2, p.scale_log2);
-  const int G = gridDim.x, c = blockIdx.x;
   uint32_t units = 0, step = 0, q_it = 0;
   for (int k = 0;; ++k) {
-    const int u = unit_for_round(k, G, c);
-    if (u >= p.units_kv) break;
+    int u;
+    if (!uq.read(k, cx, SITE_UNIT, u)) return;
+    if (u < 0) break;
     const KUnit x = kv_unit(p, u);
     QWalk it;
     it.start(p, x);
@@ -1026,6 +1033,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __gri
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem_raw + C::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem_raw + C::OFF_MISC + 4);
   const KBars br{base + C::OFF_BAR, C::NQ, C::NO};
+  // as in the dQ kernel, the loader runs at most two units ahead of the
+  // softmax warpgroups (unit k + 2 waits for the end of unit k's products)
+  const UnitQueue uq{br.units0(), base + C::OFF_UNITS};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     mbar_init(br.kv_full(), 1);
@@ -1045,6 +1055,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __gri
     mbar_init(br.acc_done(), 1);
     mbar_init(br.acc_free(), SOFTMAX_THREADS);
     mbar_init(br.drain(), 1);
+    uq.init();
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
@@ -1064,11 +1075,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ra_bwd_dkdv_kernel(const __gri
   const uint32_t tmem = *tmem_holder;
   const Ctl cx{abort_flag, p.wait_limit_ns, &g_status};
   if (warp < 8) {
-    kv_softmax<D>(p, br, tmem, lse_smem, dv_smem, warp >> 2, cx);
+    kv_softmax<D>(p, br, uq, tmem, lse_smem, dv_smem, warp >> 2, cx);
   } else if (warp == WARP_LOAD) {
-    kv_loader<D>(p, br, base, lse_smem, dv_smem, cx);
+    kv_loader<D>(p, br, uq, base, lse_smem, dv_smem, cx);
   } else {
-    kv_mma<D>(p, br, base, tmem, cx);
+    kv_mma<D>(p, br, uq, base, tmem, cx);
   }
   tc_fence_before();
   __syncthreads();
@@ -1101,13 +1112,19 @@ static cudaError_t launch_bwd_d(const BwdParams& prm, int num_sms, int max_ctas,
     if (max_ctas > 0 && max_ctas < g) g = max_ctas;
     return units < g ? units : g;
   };
+  // each launch takes its units from its own work-queue counter
+  BwdParams lp = prm;
   if (prm.parts & 1) {
-    ra_bwd_dq_kernel<D><<<grid_for(prm.units_dq), NUM_THREADS, QCfg<D>::SMEM_BYTES, stream>>>(prm);
+    e = next_ticket_counter(stream, &lp.tickets_dq);
+    if (e != cudaSuccess) return e;
+    ra_bwd_dq_kernel<D><<<grid_for(prm.units_dq), NUM_THREADS, QCfg<D>::SMEM_BYTES, stream>>>(lp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (prm.parts & 2) {
-    ra_bwd_dkdv_kernel<D><<<grid_for(prm.units_kv), NUM_THREADS, KCfg<D>::SMEM_BYTES, stream>>>(prm);
+    e = next_ticket_counter(stream, &lp.tickets_kv);
+    if (e != cudaSuccess) return e;
+    ra_bwd_dkdv_kernel<D><<<grid_for(prm.units_kv), NUM_THREADS, KCfg<D>::SMEM_BYTES, stream>>>(lp);
     e = cudaGetLastError();
   }
   return e;

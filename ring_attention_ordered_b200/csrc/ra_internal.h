@@ -93,6 +93,10 @@ struct BwdParams {
   int tiles_per_blk;
   int units_dq;                // B * Hq * n_ring * tiles_per_blk
   int units_kv;                // B * Hkv * n_ring * tiles_per_blk
+  // work-queue counters of the two launches (set by the launcher, see
+  // next_ticket_counter)
+  unsigned int* tickets_dq;
+  unsigned int* tickets_kv;
   float scale;
   float scale_log2;
   unsigned long long wait_limit_ns;
@@ -134,10 +138,11 @@ cudaError_t current_context(CUcontext* ctx);
 // the address last found for the current context is used.
 cudaError_t symbol_address(const void* symbol, void** ptr, cudaStream_t stream);
 cudaError_t read_and_clear_status(unsigned long long* out);
-// A zeroed work-queue counter for the next forward launch on `stream`: one of
-// kTicketSlots static device counters, taken in rotation and reset by a
-// memset ordered on the stream (so launches on different streams use
-// different counters, up to kTicketSlots at a time).
+// A zeroed work-queue counter for the next launch on `stream` (forward, FP8
+// forward, each backward kernel): one of kTicketSlots static device
+// counters, taken in rotation and reset by a memset ordered on the stream
+// (so launches on different streams use different counters, up to
+// kTicketSlots at a time).
 constexpr int kTicketSlots = 64;
 cudaError_t next_ticket_counter(cudaStream_t stream, unsigned int** counter);
 
