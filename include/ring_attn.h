@@ -23,8 +23,12 @@
  *     explanation that ring_attn_last_error() returns (per host thread).
  *   - The library holds no device allocation of its own except static
  *     device variables of the module: three status words per device (bf16
- *     forward, backward and FP8 forward kernels) and the fixed 4 MiB array
- *     of ring_attn_bwd_noalloc.
+ *     forward, backward and FP8 forward kernels), the fixed 4 MiB array of
+ *     ring_attn_bwd_noalloc, and 64 work-queue counters.  Each kernel launch
+ *     (one per forward call, two per backward call) takes the next counter
+ *     in rotation and zeroes it with a memset ordered on `stream`, so up to
+ *     64 launches may be in flight on different streams at once, and CUDA
+ *     graph replays start from zero.
  *   - Contexts: a call runs in the calling thread's current CUDA context,
  *     the device's primary context or one the caller created (cuCtxCreate),
  *     and `stream` must belong to that context.  A thread with no current
