@@ -353,8 +353,9 @@ ra_status ring_attn_check_status(ra_stream_t stream);
  * (nanoseconds; default 5e9).  0 restores the default.  Process-wide. */
 ra_status ring_attn_set_wait_limit_ns(uint64_t ns);
 
-/* Cap on the number of persistent CTAs of the forward kernels (0 = one per
- * SM, the default).  Process-wide; used to exercise the scheduler. */
+/* Cap on the number of persistent CTAs of the forward and backward kernels
+ * (0 = one per SM, the default).  Process-wide; used to exercise the
+ * scheduler.  Results do not depend on it. */
 ra_status ring_attn_set_max_ctas(int n);
 
 /* Order in which the forward kernels' persistent CTAs (bf16 and FP8) take

@@ -34,6 +34,10 @@
 //     dK += dS^T Q accumulate in TMEM: no atomics, every gradient is written
 //     once.  Q (read early by S^T and late by dK) has three stages.
 //   P is rounded to bf16 once and that value feeds both dV and dS.
+//   The CTAs of each launch take their units from one work queue
+//   (ra_unit_queue.cuh), head by head and longest first inside a head, so
+//   they stay within about one unit of each other and share K/V (dQ kernel)
+//   or Q/dO tiles (dK/dV kernel) in L2.
 //   Every mbarrier wait is bounded (ra_sync.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
